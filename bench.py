@@ -1,0 +1,377 @@
+"""Benchmark of the PBD window-attention path on B200.
+
+One step = one PBD decode step of the workload: for every layer, the window K/V append and
+the window attention (``la_pbd_step`` through the C ABI). Default workload: the single-image
+decode step (batch 1, 36 layers, prefix 1024 = 256 visual + 768 text/box tokens, window 6,
+16 query / 2 KV heads, d = 128, 1% of K channels x8), seed 1.
+
+Timing: inputs resident in HBM, several full copies of the workload rotated so that every step
+reads data that is not in L2 (working set > 2 x L2); the step is captured in a CUDA graph; W
+untimed warm-up steps; K timed steps between CUDA events on the launching stream with a
+barrier and synchronize on both sides; max over ranks. `e2e` repeats the measurement through
+the same C ABI with the step's inputs (Q, new K/V of every layer) copied from pinned host
+memory and the output copied back inside the timed region.
+
+Multi-GPU: replicas only (each rank runs its own independent batch; no collective on the data
+path; the timing uses one max-reduction).
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "PBD window-steps/sec and achieved HBM GB/s (% of B200 peak) vs prefix length"
+UNIT = "window-steps/s"
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- setup
+def build_device_inputs(wi, copies, device):
+    """Stack every layer's tensors and make `copies` independent copies on the device."""
+    import torch
+    L = len(wi.layers)
+    stack = lambda name: torch.stack([getattr(li, name) for li in wi.layers])  # noqa: E731
+    host = {n: stack(n) for n in ("q", "k_cache", "v_cache", "k_new", "v_new")}
+    dev = []
+    for c in range(copies):
+        d = {n: t.to(device) for n, t in host.items()}
+        d["out"] = torch.empty_like(d["q"])
+        dev.append(d)
+    seq = wi.seq_lens.to(device)
+    return host, dev, seq, L
+
+
+def run_step(bmw, cfg, d, seq, W, ws, L):
+    for layer in range(L):
+        bmw.la_pbd_step(cfg, d["q"][layer], d["k_new"][layer], d["v_new"][layer],
+                        d["k_cache"][layer], d["v_cache"][layer], seq, W, d["out"][layer], ws)
+
+
+def run_attn_only(bmw, cfg, d, seq, W, ws, L):
+    for layer in range(L):
+        bmw.la_pbd_attn(cfg, d["q"][layer], d["k_cache"][layer], d["v_cache"][layer], seq, W,
+                        d["out"][layer], ws)
+
+
+def capture(torch, fn):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm (kernel attributes, tensor-map encoder)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graphs(torch, graphs, steps, warmup, barrier):
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    end.record()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
+    wi = workloads.generate(wl)
+    B, W = wl.batch, wl.window
+    per_copy = (2 * wi.layers[0].k_cache.numel() * 2 + 3 * wi.layers[0].q.numel() * 2) * len(wi.layers)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(2, min(args.max_copies, math.ceil(2.5 * l2 / max(per_copy, 1))))
+    host, dev, seq, L = build_device_inputs(wi, copies, device)
+    cfg = bmw.Config.make(B, wl.num_q_heads, wl.num_kv_heads, wi.max_seq, algo=args.algo)
+    ws = bmw.Workspace(cfg, W, device=device)
+
+    step_graphs = [capture(torch, lambda d=d: run_step(bmw, cfg, d, seq, W, ws, L)) for d in dev]
+    steps, warmup = args.steps, args.warmup
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    ms = time_graphs(torch, step_graphs, steps, warmup, barrier)
+    clk = clocks.stop()
+    ms = max_over_ranks(ms)
+    ms_per_step = ms / steps
+    value = world * B * steps / (ms / 1e3)
+
+    # Dominant kernel: the attention call of one layer (attention + split merge), timed alone
+    # over the same rotating copies.
+    attn_graphs = [capture(torch, lambda d=d: run_attn_only(bmw, cfg, d, seq, W, ws, L)) for d in dev]
+    reps = max(steps, 20)
+    ms_attn = time_graphs(torch, attn_graphs, reps, warmup, barrier)
+    ms_attn = max_over_ranks(ms_attn)
+    launch_us = ms_attn * 1e3 / (reps * L)
+    alg_bytes = workloads.algorithmic_bytes(wi.seq_lens.tolist(), W, wl.num_q_heads,
+                                            wl.num_kv_heads, wl.head_dim)
+    achieved = alg_bytes / (launch_us * 1e-6) / 1e9
+    step_bytes = L * (alg_bytes + workloads.append_bytes(B, W, wl.num_kv_heads, wl.head_dim))
+    if bmw.la_pbd_check(ws) != 0:
+        raise RuntimeError("device-side status not OK after the benchmark")
+
+    # End to end through the same API: inputs from pinned host memory, output back to host.
+    e2e = None
+    if not args.no_e2e:
+        h_in = {n: host[n].pin_memory() for n in ("q", "k_new", "v_new")}
+        h_out = torch.empty_like(host["q"]).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = h_out.numel() * h_out.element_size()
+        for i in range(warmup):
+            d = dev[i % copies]
+            for n in h_in:
+                d[n].copy_(h_in[n], non_blocking=True)
+            step_graphs[i % copies].replay()
+            h_out.copy_(d["out"], non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            d = dev[i % copies]
+            for n in h_in:
+                d[n].copy_(h_in[n], non_blocking=True)
+            step_graphs[i % copies].replay()
+            h_out.copy_(d["out"], non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": world * B * steps / (ms_e2e / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ms_e2e / steps}
+    del step_graphs, attn_graphs
+    return {
+        "wi": wi, "ms_per_step": ms_per_step, "value": value, "clocks": clk,
+        "launch_us": launch_us, "alg_bytes": alg_bytes, "achieved_gbs": achieved,
+        "step_bytes": step_bytes, "copies": copies, "e2e": e2e, "layers": L,
+        "launches_per_step": L * 3,
+    }
+
+
+def cpu_baseline(wl, budget_s):
+    """The fp64 oracle on a bounded sample of the workload (whole layers)."""
+    import numpy as np  # noqa: F401
+    import oracle
+    wi = workloads.generate(wl, layers=min(wl.layers, 4))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        li = wi.layers[done % len(wi.layers)]
+        oracle.pbd_step(li.q, li.k_cache, li.v_cache, li.k_new, li.v_new, wi.seq_lens, wl.scale)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= 4 * wl.layers:
+            break
+    per_layer = el / done
+    value = wl.batch / (per_layer * wl.layers)
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} layer calls of the {wl.name} workload ({el:.1f} s), scaled to "
+                      f"{wl.layers}-layer steps; numpy fp64, all host threads"}
+
+
+def workload_label(wl):
+    return {"workload": wl.name, "batch": wl.batch, "layers": wl.layers,
+            "prefix": wl.prefix if wl.prefix is not None else "ragged U{512..4096}+U{1..5}",
+            "window": wl.window, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
+            "head_dim": wl.head_dim, "seed": wl.seed}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="single_image", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--algo", type=int, default=0, help="0 auto, 1 tcgen05, 2 CUDA cores")
+    ap.add_argument("--sweep", default="max_context,max_context_w1,ragged,long",
+                    help="extra workloads measured for the prefix-length sweep ('' for none)")
+    ap.add_argument("--max-copies", type=int, default=16)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = workloads.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = cpu_baseline(wl, args.cpu_budget)
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * wl.batch / cb["value"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": workload_label(wl), "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    import block_masked_window_b200 as bmw
+    bmw.load()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        device = torch.device("cuda", local_rank)
+
+        def barrier():
+            dist.barrier()
+
+        def max_over_ranks(x):
+            t = torch.tensor([x], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+    else:
+        device = torch.device("cuda", 0)
+        torch.cuda.set_device(0)
+        barrier = lambda: None  # noqa: E731
+        max_over_ranks = lambda x: x  # noqa: E731
+
+    res = measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks)
+    peak, peak_kind = measured_peaks()
+    sweep = []
+    for name in [s for s in args.sweep.split(",") if s]:
+        swl = workloads.WORKLOADS[name]
+        sargs = argparse.Namespace(**vars(args))
+        sargs.steps = max(10, min(args.steps, 20))
+        sargs.no_e2e = True
+        r = measure(sargs, rank, world, device, bmw, torch, swl, barrier, max_over_ranks)
+        sweep.append({
+            "workload": name, "prefix": swl.prefix if swl.prefix is not None else "ragged",
+            "batch": swl.batch, "window": swl.window, "layers": swl.layers,
+            "window_steps_per_s": r["value"], "ms_per_step": r["ms_per_step"],
+            "attn_launch_us": r["launch_us"], "attn_bytes_per_launch": r["alg_bytes"],
+            "achieved_gbs": r["achieved_gbs"], "frac_of_measured_hbm": r["achieved_gbs"] / peak,
+            "frac_of_8tbs": r["achieved_gbs"] / 8000.0,
+        })
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    cb = cpu_baseline(wl, args.cpu_budget) if world == 1 else None
+    wi = res["wi"]
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V, per the workload recipe)",
+        "config": dict(workload_label(wl), **{
+            "parallelism": f"replicas x{world}", "l2": f"inputs > L2: {res['copies']} rotating copies",
+            "graph": "CUDA graph per step", "algo": args.algo}),
+        "roofline": {"bound": "hbm", "achieved": res["achieved_gbs"], "peak": peak,
+                     "unit": "GB/s", "frac": res["achieved_gbs"] / peak,
+                     "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "la_pbd_attn (split-KV attention + merge), one layer",
+                     "bytes_per_launch": res["alg_bytes"], "launch_us": res["launch_us"]},
+        "gpu_launches": res["launches_per_step"] * args.steps,
+        "e2e": res["e2e"], "clocks": res["clocks"], "cpu_baseline": cb,
+        "step_bytes": res["step_bytes"],
+        "step_gbs": res["step_bytes"] / (res["ms_per_step"] * 1e-3) / 1e9,
+        "sweep": sweep,
+    }
+    print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,215 @@
+"""Python binding of ``libla_pbd.so``, the B200 PBD window-attention library.
+
+Argument marshalling only: every step of the computation runs in the library's CUDA kernels
+(see ``include/la_pbd.h`` for the C ABI). The functions take torch CUDA tensors for device
+memory and use torch's current CUDA stream; they never fall back to another implementation:
+if the shared library is missing or fails to load, they raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+__all__ = [
+    "LA_MASK_PBD", "LA_MASK_CAUSAL_WINDOW", "LA_ALGO_AUTO", "LA_ALGO_TCGEN05", "LA_ALGO_SIMT",
+    "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
+    "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
+    "la_pbd_step", "la_pbd_check", "Workspace", "EXPORTED_SYMBOLS",
+]
+
+LA_MASK_PBD = 0
+LA_MASK_CAUSAL_WINDOW = 1
+LA_ALGO_AUTO = 0
+LA_ALGO_TCGEN05 = 1
+LA_ALGO_SIMT = 2
+
+LA_OK = 0
+STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
+                3: "LA_ERR_WORKSPACE", 4: "LA_ERR_CUDA", 5: "LA_ERR_SEQ_OVERFLOW",
+                6: "LA_ERR_TIMEOUT"}
+
+EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
+                    "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
+                    "la_pbd_check"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB: Optional[ctypes.CDLL] = None
+
+
+class LaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} "
+                         f"({la_status_string(status) if _LIB else ''})")
+
+
+class Config(ctypes.Structure):
+    """Mirror of ``la_pbd_cfg``."""
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("max_seq", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("mask_mode", ctypes.c_int32), ("algo", ctypes.c_int32)]
+
+    @classmethod
+    def make(cls, batch, num_q_heads, num_kv_heads, max_seq, head_dim=128, scale=None,
+             mask_mode=LA_MASK_PBD, algo=LA_ALGO_AUTO) -> "Config":
+        if scale is None:
+            scale = 1.0 / math.sqrt(head_dim)
+        return cls(batch, num_q_heads, num_kv_heads, head_dim, max_seq, scale, mask_mode, algo)
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libla_pbd.so")
+
+
+def load() -> ctypes.CDLL:
+    """Load the shared library (raises if it has not been built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m block_masked_window_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    cfgp = ctypes.POINTER(Config)
+    lib.la_version.restype = i32
+    lib.la_version.argtypes = []
+    lib.la_status_string.restype = ctypes.c_char_p
+    lib.la_status_string.argtypes = [i32]
+    lib.la_pbd_workspace_bytes.restype = sz
+    lib.la_pbd_workspace_bytes.argtypes = [cfgp, i32]
+    lib.la_pbd_workspace_init.restype = i32
+    lib.la_pbd_workspace_init.argtypes = [vp, sz, vp]
+    lib.la_kv_append.restype = i32
+    lib.la_kv_append.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp]
+    lib.la_pbd_attn.restype = i32
+    lib.la_pbd_attn.argtypes = [cfgp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+    lib.la_pbd_step.restype = i32
+    lib.la_pbd_step.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+    lib.la_pbd_check.restype = i32
+    lib.la_pbd_check.argtypes = [vp, vp]
+    _LIB = lib
+    return lib
+
+
+def la_version() -> int:
+    return load().la_version()
+
+
+def la_status_string(status: int) -> str:
+    return load().la_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != LA_OK:
+        raise LaError(status, where)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    if stream is not None:
+        return int(stream) if isinstance(stream, int) else int(stream.cuda_stream)
+    import torch
+    return int(torch.cuda.current_stream().cuda_stream)
+
+
+def _check_tensor(t, name, dtype_name, shape=None):
+    import torch
+    dt = {"bf16": torch.bfloat16, "i32": torch.int32}[dtype_name]
+    if t.dtype != dt:
+        raise TypeError(f"{name}: expected {dtype_name}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def la_pbd_workspace_bytes(cfg: Config, window_len: int) -> int:
+    return int(load().la_pbd_workspace_bytes(ctypes.byref(cfg), int(window_len)))
+
+
+def la_pbd_workspace_init(workspace, stream=None) -> None:
+    _check(load().la_pbd_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "la_pbd_workspace_init")
+
+
+class Workspace:
+    """A device workspace sized by ``la_pbd_workspace_bytes`` (allocated through torch)."""
+
+    def __init__(self, cfg: Config, window_len: int, device=None):
+        import torch
+        n = la_pbd_workspace_bytes(cfg, window_len)
+        if n == 0:
+            raise LaError(2, "la_pbd_workspace_bytes")
+        self.nbytes = n
+        self.buf = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
+        off = (-self.buf.data_ptr()) % 256
+        self.tensor = self.buf[off:off + n]
+        la_pbd_workspace_init(self.tensor)
+
+    def data_ptr(self) -> int:
+        return int(self.tensor.data_ptr())
+
+
+def _shapes(cfg: Config, W: int):
+    B, Hq, Hkv, D, S = cfg.batch, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, cfg.max_seq
+    return (B, W, Hq, D), (B, Hkv, S, D), (B, W, Hkv, D)
+
+
+def la_kv_append(cfg: Config, k_new, v_new, k_cache, v_cache, seq_lens, window_len: int,
+                 stream=None) -> None:
+    W = int(window_len)
+    _, cache_shape, new_shape = _shapes(cfg, W)
+    _check_tensor(k_new, "k_new", "bf16", new_shape)
+    _check_tensor(v_new, "v_new", "bf16", new_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check(load().la_kv_append(ctypes.byref(cfg), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                               _ptr(v_cache), _ptr(seq_lens), W, _stream(stream)),
+           "la_kv_append")
+
+
+def la_pbd_attn(cfg: Config, q, k_cache, v_cache, seq_lens, window_len: int, out,
+                workspace: Workspace, stream=None) -> None:
+    W = int(window_len)
+    q_shape, cache_shape, _ = _shapes(cfg, W)
+    _check_tensor(q, "q", "bf16", q_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check_tensor(out, "out", "bf16", q_shape)
+    _check(load().la_pbd_attn(ctypes.byref(cfg), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                              _ptr(seq_lens), W, _ptr(out), workspace.data_ptr(),
+                              workspace.nbytes, _stream(stream)), "la_pbd_attn")
+
+
+def la_pbd_step(cfg: Config, q, k_new, v_new, k_cache, v_cache, seq_lens, window_len: int, out,
+                workspace: Workspace, stream=None) -> None:
+    W = int(window_len)
+    q_shape, cache_shape, new_shape = _shapes(cfg, W)
+    _check_tensor(q, "q", "bf16", q_shape)
+    _check_tensor(k_new, "k_new", "bf16", new_shape)
+    _check_tensor(v_new, "v_new", "bf16", new_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check_tensor(out, "out", "bf16", q_shape)
+    _check(load().la_pbd_step(ctypes.byref(cfg), _ptr(q), _ptr(k_new), _ptr(v_new),
+                              _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), W, _ptr(out),
+                              workspace.data_ptr(), workspace.nbytes, _stream(stream)),
+           "la_pbd_step")
+
+
+def la_pbd_check(workspace: Workspace, stream=None) -> int:
+    """Synchronise and return the sticky device status (0 = LA_OK); clears it."""
+    return int(load().la_pbd_check(workspace.data_ptr(), _stream(stream)))

@@ -1,0 +1,224 @@
+// C ABI of the PBD window-attention library (declared in include/la_pbd.h): argument
+// validation, workspace sizing, kernel selection and launch. Nothing here allocates device
+// memory or synchronises, except la_pbd_check.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/la_pbd.h"
+#include "pbd_common.cuh"
+#include "pbd_kernels.h"
+#include "tma_util.h"
+
+namespace {
+
+using la::Problem;
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+std::mutex g_mu;
+
+cudaError_t sm_count(int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    g_sm_count[dev] = n;
+  }
+  *out = g_sm_count[dev];
+  return cudaSuccess;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+la_status check_cfg(const la_pbd_cfg* cfg, int32_t W) {
+  if (!cfg) return LA_ERR_INVALID_ARG;
+  if (cfg->batch < 1 || cfg->batch > la::kMaxBatch) return LA_ERR_INVALID_ARG;
+  if (cfg->num_kv_heads < 1 || cfg->num_q_heads < 1) return LA_ERR_INVALID_ARG;
+  if (cfg->max_seq < 1) return LA_ERR_INVALID_ARG;
+  if (!std::isfinite(cfg->scale)) return LA_ERR_INVALID_ARG;
+  if (W < 1 || W > la::kMaxWindow) return LA_ERR_INVALID_ARG;
+  if (cfg->mask_mode != LA_MASK_PBD && cfg->mask_mode != LA_MASK_CAUSAL_WINDOW)
+    return LA_ERR_INVALID_ARG;
+  if (cfg->algo != LA_ALGO_AUTO && cfg->algo != LA_ALGO_TCGEN05 && cfg->algo != LA_ALGO_SIMT)
+    return LA_ERR_INVALID_ARG;
+  if (cfg->head_dim != la::kHeadDim) return LA_ERR_UNSUPPORTED;
+  if (cfg->num_q_heads % cfg->num_kv_heads != 0) return LA_ERR_UNSUPPORTED;
+  // Per-head prefix sums and TMA row coordinates are int32: B * Hkv * S_max < 2^31.
+  if ((long long)cfg->batch * cfg->num_kv_heads * cfg->max_seq >= (1LL << 31))
+    return LA_ERR_UNSUPPORTED;
+  const long long R = (long long)W * (cfg->num_q_heads / cfg->num_kv_heads);
+  if (R > 128) return LA_ERR_UNSUPPORTED;
+  if (cfg->algo == LA_ALGO_TCGEN05 && R > 64) return LA_ERR_UNSUPPORTED;
+  return LA_OK;
+}
+
+// Kernel choice for a validated configuration.
+int pick_algo(const la_pbd_cfg* cfg, int R) {
+  if (cfg->algo != LA_ALGO_AUTO) return cfg->algo;
+  return (R <= 64) ? LA_ALGO_TCGEN05 : LA_ALGO_SIMT;
+}
+
+size_t slots_for(const la_pbd_cfg* cfg, int sms) {
+  return (size_t)sms * la::kMaxCtasPerSm + (size_t)cfg->batch * cfg->num_kv_heads;
+}
+
+la_status fill_problem(const la_pbd_cfg* cfg, int32_t W, Problem* p) {
+  std::memset(p, 0, sizeof(*p));
+  p->B = cfg->batch;
+  p->Hq = cfg->num_q_heads;
+  p->Hkv = cfg->num_kv_heads;
+  p->G = cfg->num_q_heads / cfg->num_kv_heads;
+  p->W = W;
+  p->S = cfg->max_seq;
+  p->R = W * p->G;
+  p->rows_pad = la::round_up(p->R, 16);
+  p->mask_mode = cfg->mask_mode;
+  p->scale_log2 = cfg->scale * 1.4426950408889634f;
+  return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t la_version(void) { return 100; }
+
+const char* la_status_string(la_status s) {
+  switch (s) {
+    case LA_OK: return "ok";
+    case LA_ERR_INVALID_ARG: return "invalid argument";
+    case LA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LA_ERR_CUDA: return "CUDA error";
+    case LA_ERR_SEQ_OVERFLOW: return "a sequence had seq_len < 0 or seq_len + window > max_seq";
+    case LA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t la_pbd_workspace_bytes(const la_pbd_cfg* cfg, int32_t W) {
+  if (check_cfg(cfg, W) != LA_OK) return 0;
+  int sms = 0;
+  if (sm_count(&sms) != cudaSuccess) return 0;
+  const int G = cfg->num_q_heads / cfg->num_kv_heads;
+  const int rows_pad = la::round_up(W * G, 16);
+  return la::kSlotsOffset + slots_for(cfg, sms) * la::slot_floats(rows_pad) * sizeof(float);
+}
+
+static la_status check_attn_args(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* seq_lens, int32_t W,
+                                 const void* out, const void* workspace,
+                                 size_t workspace_bytes) {
+  la_status st = check_cfg(cfg, W);
+  if (st != LA_OK) return st;
+  if (!q || !k_cache || !v_cache || !seq_lens || !out) return LA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(seq_lens, 4))
+    return LA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return LA_ERR_WORKSPACE;
+  const size_t need = la_pbd_workspace_bytes(cfg, W);
+  if (need == 0) return LA_ERR_CUDA;
+  if (workspace_bytes < need) return LA_ERR_WORKSPACE;
+  return LA_OK;
+}
+
+la_status la_pbd_workspace_init(void* workspace, size_t bytes, void* stream) {
+  if (!workspace || bytes < la::kSlotsOffset || !aligned(workspace, 256)) return LA_ERR_WORKSPACE;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, la::kHeaderBytes, (cudaStream_t)stream);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_kv_append(const la_pbd_cfg* cfg, const void* k_new, const void* v_new, void* k_cache,
+                       void* v_cache, const int32_t* seq_lens, int32_t W, void* stream) {
+  la_status st = check_cfg(cfg, W);
+  if (st != LA_OK) return st;
+  if (!k_new || !v_new || !k_cache || !v_cache || !seq_lens) return LA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16) || !aligned(seq_lens, 4))
+    return LA_ERR_INVALID_ARG;
+  cudaError_t e = la::launch_kv_append(k_new, v_new, k_cache, v_cache, seq_lens, cfg->batch, W,
+                                       cfg->num_kv_heads, cfg->max_seq, (cudaStream_t)stream);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, int32_t W, void* out,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+
+  Problem p;
+  fill_problem(cfg, W, &p);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seq_lens = seq_lens;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  char* ws = static_cast<char*>(workspace);
+  p.hdr = reinterpret_cast<la::WsHeader*>(ws);
+  p.pre_g = reinterpret_cast<int*>(ws + la::kPrefixOffset);
+  p.partials = reinterpret_cast<float*>(ws + la::kSlotsOffset);
+
+  int sms = 0;
+  if (sm_count(&sms) != cudaSuccess) return LA_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  const int algo = pick_algo(cfg, p.R);
+  if (algo == LA_ALGO_TCGEN05) {
+    la::TmaMaps maps;
+    if (la::make_tma_maps(p, &maps) != cudaSuccess) return LA_ERR_CUDA;
+    p.num_ctas = sms * la::tc_ctas_per_sm();
+    p.c_min = la::tc_min_chunk();
+    e = la::launch_attn_tc(p, &maps.k, &maps.v, &maps.q, s);
+  } else {
+    int per_sm = 0;
+    e = la::simt_max_ctas_per_sm(p.R, p.B, &per_sm);
+    if (e != cudaSuccess) return LA_ERR_CUDA;
+    if (per_sm < 1) return LA_ERR_UNSUPPORTED;
+    if (per_sm > la::kMaxCtasPerSm) per_sm = la::kMaxCtasPerSm;
+    p.num_ctas = sms * per_sm;
+    p.c_min = 32;
+    e = la::launch_attn_simt(p, s);
+  }
+  if (e != cudaSuccess) return LA_ERR_CUDA;
+  e = la::launch_combine(p, s);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new, const void* v_new,
+                      void* k_cache, void* v_cache, const int32_t* seq_lens, int32_t W,
+                      void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  // Validate both halves before enqueuing anything.
+  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return LA_ERR_INVALID_ARG;
+  st = la_kv_append(cfg, k_new, v_new, k_cache, v_cache, seq_lens, W, stream);
+  if (st != LA_OK) return st;
+  return la_pbd_attn(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, workspace_bytes,
+                     stream);
+}
+
+la_status la_pbd_check(void* workspace, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return LA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t err = 0;
+  cudaError_t e = cudaMemcpyAsync(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return LA_ERR_CUDA;
+  if (err & la::kErrTimeout) return LA_ERR_TIMEOUT;
+  if (err & la::kErrSeqOverflow) return LA_ERR_SEQ_OVERFLOW;
+  return LA_OK;
+}
+
+}  // extern "C"

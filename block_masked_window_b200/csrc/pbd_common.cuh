@@ -1,0 +1,187 @@
+// Shared device-side pieces of the PBD window-attention kernels: constants, the workspace
+// header, the partial-result slot layout and the flattened split-KV work plan.
+//
+// Work plan ("stream-K" over tokens). Sequence s = b * Hkv + h (batch b, KV head h) has
+// N_b = P_b + W visible keys (0 if P_b is invalid). All sequences are laid end to end in one
+// flattened token stream of length T = Hkv * sum_b N_b. CTA c of a grid of G CTAs owns tokens
+// [c*C, (c+1)*C) with C = max(c_min, ceil(T / G)), so every CTA gets the same number of keys
+// whatever the mix of prefix lengths. The part of a sequence that falls in one CTA is a
+// segment; a CTA that holds a whole sequence writes its final output directly, every other
+// segment writes an (m, l, acc) partial to slot c + s, and the combine kernel merges them.
+// Slot c + s is unique because CTAs and sequences advance together along the stream.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace la {
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxBatch = 4096;
+constexpr int kMaxWindow = 16;
+constexpr int kHeaderBytes = 256;
+
+// Sticky error bits in the workspace header (first 32-bit word).
+constexpr uint32_t kErrSeqOverflow = 1u;
+constexpr uint32_t kErrTimeout = 2u;
+
+struct WsHeader {
+  uint32_t err;
+  uint32_t pad[63];
+};
+
+// Launch-wide parameters shared by the attention and combine kernels.
+struct Problem {
+  const __nv_bfloat16* q;       // [B, W, Hq, D]
+  const __nv_bfloat16* k;       // [B, Hkv, S, D]
+  const __nv_bfloat16* v;       // [B, Hkv, S, D]
+  const int32_t* seq_lens;      // [B]
+  __nv_bfloat16* out;           // [B, W, Hq, D]
+  float* partials;              // slots, see slot_floats
+  WsHeader* hdr;
+  int* pre_g;                   // [B+1] prefix sums of N_b, written by attention CTA 0
+  int B, Hq, Hkv, G, W, S;      // G = Hq / Hkv
+  int R;                        // rows per sequence = W * G
+  int rows_pad;                 // R rounded up to 16: rows per partial slot
+  int mask_mode;                // 0 = PBD window, 1 = causal window
+  int num_ctas;                 // grid size of the attention kernel (fixes the chunk size)
+  int c_min;                    // minimum tokens per CTA
+  float scale_log2;             // scale * log2(e)
+};
+
+__host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+__host__ __device__ inline size_t slot_floats(int rows_pad) {
+  return (size_t)rows_pad * (kHeadDim + 2);
+}
+// Slot layout: m[rows_pad] (log2 domain), l[rows_pad], acc[rows_pad][D].
+__device__ inline float* slot_ptr(const Problem& p, int slot) {
+  return p.partials + (size_t)slot * slot_floats(p.rows_pad);
+}
+
+// Visible keys of sequence b (0 marks an invalid prefix length).
+__device__ inline int visible_len(const Problem& p, int b) {
+  int P = __ldg(p.seq_lens + b);
+  if (P < 0 || (long long)P + p.W > (long long)p.S) return 0;
+  return P + p.W;
+}
+
+// Block-wide prefix sum of N_b into pre[0..B] (pre[0] = 0, pre[b+1] = N_0 + ... + N_b).
+// Every thread of the block must call it. `warp_tot` needs one int per warp (<= 32).
+__device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, wid = tid >> 5;
+  const int nwarps = (nthr + 31) >> 5;
+  int carry = 0;
+  if (tid == 0) pre[0] = 0;
+  for (int base = 0; base < p.B; base += nthr) {
+    int b = base + tid;
+    int x = (b < p.B) ? visible_len(p, b) : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int t = (lane < nwarps) ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      if (lane < nwarps) warp_tot[lane] = t;  // inclusive over warps
+    }
+    __syncthreads();
+    int add = carry + (wid > 0 ? warp_tot[wid - 1] : 0);
+    if (b < p.B) pre[b + 1] = x + add;
+    carry += warp_tot[nwarps - 1];
+    __syncthreads();
+  }
+}
+
+// Chunk size C from the total T (identical in every kernel that uses the plan).
+__device__ inline long long plan_chunk(const Problem& p, long long T) {
+  long long c = (T + p.num_ctas - 1) / p.num_ctas;
+  return c < p.c_min ? (long long)p.c_min : c;
+}
+
+// Largest b with Hkv * pre[b] <= pos (pos < T). Never returns a zero-length sequence.
+__device__ inline int plan_find_batch(const Problem& p, const int* pre, long long pos) {
+  int lo = 0, hi = p.B - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if ((long long)p.Hkv * pre[mid] <= pos) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+struct Segment {
+  int b, h;        // batch, KV head
+  int n;           // visible keys of the sequence (N_b)
+  int j0, j1;      // key range of this segment, 0 <= j0 < j1 <= n
+  bool whole;      // the segment is the whole sequence
+  int slot;        // partial slot (when !whole)
+};
+
+// Iterator over the segments of CTA `c`.
+struct SegmentIter {
+  long long pos, end;
+  int b, h;
+  __device__ bool next(const Problem& p, const int* pre, int c, Segment& sg) {
+    while (pos < end) {
+      int n = pre[b + 1] - pre[b];
+      long long s0 = (long long)p.Hkv * pre[b] + (long long)h * n;
+      if (n == 0 || pos >= s0 + n) {  // advance to the next sequence
+        if (++h == p.Hkv) { h = 0; ++b; }
+        continue;
+      }
+      long long lo = pos, hi = (end < s0 + n) ? end : s0 + n;
+      sg.b = b; sg.h = h; sg.n = n;
+      sg.j0 = (int)(lo - s0); sg.j1 = (int)(hi - s0);
+      sg.whole = (sg.j0 == 0 && sg.j1 == n);
+      sg.slot = c + b * p.Hkv + h;
+      pos = hi;
+      return true;
+    }
+    return false;
+  }
+};
+
+__device__ inline SegmentIter plan_begin(const Problem& p, const int* pre, int c, long long C,
+                                         long long T) {
+  SegmentIter it;
+  it.pos = (long long)c * C;
+  it.end = it.pos + C < T ? it.pos + C : T;
+  it.b = 0; it.h = 0;
+  if (it.pos < T) {
+    int b = plan_find_batch(p, pre, it.pos);
+    int n = pre[b + 1] - pre[b];
+    long long off = it.pos - (long long)p.Hkv * pre[b];
+    it.b = b;
+    it.h = n > 0 ? (int)(off / n) : 0;
+    if (it.h >= p.Hkv) it.h = p.Hkv - 1;
+  }
+  return it;
+}
+
+// Output row r of sequence (b, h): window row i = r / G, query head h*G + r % G.
+__device__ inline size_t out_row_offset(const Problem& p, int b, int h, int r) {
+  int i = r / p.G, g = r - i * p.G;
+  return (((size_t)b * p.W + i) * p.Hq + (size_t)h * p.G + g) * kHeadDim;
+}
+
+// Number of keys visible to window row i in a sequence of n = P + W visible keys.
+__device__ inline int row_limit(const Problem& p, int n, int r) {
+  if (p.mask_mode == 0) return n;
+  int i = r / p.G;
+  return n - p.W + i + 1;
+}
+
+__device__ inline float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+}  // namespace la

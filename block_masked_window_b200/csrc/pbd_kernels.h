@@ -1,0 +1,35 @@
+// Host-side launchers of the PBD kernels (internal to the library; the public C ABI is
+// include/la_pbd.h).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "pbd_common.cuh"
+
+namespace la {
+
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int32_t* seq_lens, int B, int W, int Hkv, int S,
+                             cudaStream_t stream);
+
+// CUDA-core split-KV attention (any R = W * G <= 128).
+int simt_rows_per_thread(int R);
+size_t simt_smem_bytes(int R, int B);
+cudaError_t simt_max_ctas_per_sm(int R, int B, int* ctas);
+cudaError_t launch_attn_simt(const Problem& p, cudaStream_t stream);
+
+// tcgen05 + TMA split-KV attention (R <= 64).
+size_t tc_smem_bytes(int B);
+cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tmap_v,
+                           const void* tmap_q, cudaStream_t stream);
+
+// Merge of the per-split partials into the bf16 output.
+cudaError_t launch_combine(const Problem& p, cudaStream_t stream);
+
+// Workspace carve-up shared by the launchers and the C ABI.
+constexpr size_t kPrefixOffset = kHeaderBytes;                               // int[B+1]
+constexpr size_t kPrefixBytes = ((size_t)(kMaxBatch + 1) * 4 + 255) / 256 * 256;
+constexpr size_t kSlotsOffset = kPrefixOffset + kPrefixBytes;
+constexpr int kMaxCtasPerSm = 4;
+
+}  // namespace la

@@ -1,0 +1,143 @@
+/*
+ * la_pbd.h -- C ABI of the B200 (sm_100a) Parallel Box Decoding window-attention library.
+ *
+ * What the library computes
+ * -------------------------
+ * One PBD decode step of LocateAnything-3B attends a window of W query tokens (the last
+ * accepted token plus 5 <text_mask> tokens, so W = 6; W = 1 is plain next-token decoding)
+ * over the decoder's KV cache. Inside the window attention is bidirectional; toward the
+ * prefix it is causal, so every window row sees cache rows [0, P_b + W) of its sequence and
+ * nothing beyond (LocateAnything-3B for RK3588 model card, "How it differs from the
+ * original", item 1). The decoder is Qwen2.5-3B: 36 layers, K/V tensors of shape
+ * [1, 2, seq, 128] per layer (LocateAnything-3B ONNX WebGPU INT4 model card, "KV-cache graph
+ * for in-browser use"), hidden size 2048 (same card, "Why this repo exists"), so 16 query
+ * heads share 2 KV heads; bf16 throughout ("LocateAnything-3B on a 12 GB RTX 4000 Ada",
+ * "Architecture footprint").
+ *
+ * For sequence b, query head h, window row i (position P_b + i):
+ *   s_j  = scale * <q[b,i,h,:], k[b, h / (Hq/Hkv), j, :]>          j in [0, P_b + W)
+ *   out[b,i,h,:] = sum_j softmax_j(s) * v[b, h / (Hq/Hkv), j, :]
+ * computed with bf16 inputs, fp32 accumulation, bf16 (round-to-nearest-even) output.
+ *
+ * Layouts (all row-major, contiguous, device memory unless stated)
+ *   q, out         bf16 [B, W, Hq, D]
+ *   k_cache,v_cache bf16 [B, Hkv, S_max, D]   one row = D * 2 = 256 bytes, 16-byte aligned
+ *   k_new, v_new   bf16 [B, W, Hkv, D]       window keys/values, RoPE already applied
+ *   seq_lens       int32 [B]                 committed prefix length P_b of each sequence
+ *
+ * Ownership: the caller owns every buffer. The compute entry points never allocate, free or
+ * synchronise; they enqueue work on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ * default stream) and return. They are reentrant. Run la_kv_append before la_pbd_attn on the
+ * same stream (or use la_pbd_step, which does both).
+ *
+ * Errors: static arguments are checked on the host and reported synchronously (nothing is
+ * enqueued on error). Per-sequence errors found on the device (seq_lens[b] < 0 or
+ * seq_lens[b] + W > max_seq) never fault: that sequence's output rows are written as zeros,
+ * its cache is left untouched, and a sticky flag is raised in the workspace header, read and
+ * cleared by la_pbd_check. Kernel launch failures map to LA_ERR_CUDA.
+ */
+#ifndef LA_PBD_H_
+#define LA_PBD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum la_status {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer               */
+  LA_ERR_UNSUPPORTED = 2,   /* head_dim != 128, Hq % Hkv != 0, W * Hq/Hkv too large ... */
+  LA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than la_pbd_workspace_bytes */
+  LA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed                        */
+  LA_ERR_SEQ_OVERFLOW = 5,  /* (la_pbd_check) a sequence had P < 0 or P + W > max_seq   */
+  LA_ERR_TIMEOUT = 6        /* (la_pbd_check) a bounded device-side wait gave up        */
+} la_status;
+
+/* Mask applied inside the window. */
+enum {
+  LA_MASK_PBD = 0,            /* bidirectional inside the window (the trained model)       */
+  LA_MASK_CAUSAL_WINDOW = 1   /* causal inside the window: row i sees [0, P_b + i]; the
+                                 RKLLM approximation (RK3588 card, item 1)                 */
+};
+
+/* Kernel selection. */
+enum {
+  LA_ALGO_AUTO = 0,      /* tensor-core kernel when supported, else CUDA cores             */
+  LA_ALGO_TCGEN05 = 1,   /* tcgen05 (TMEM accumulators) + TMA staging; W * Hq/Hkv <= 64    */
+  LA_ALGO_SIMT = 2       /* fp32 CUDA-core kernel; W * Hq/Hkv <= 128                       */
+};
+
+typedef struct la_pbd_cfg {
+  int32_t batch;         /* B >= 1, B <= 4096                                              */
+  int32_t num_q_heads;   /* Hq, a multiple of num_kv_heads                                  */
+  int32_t num_kv_heads;  /* Hkv >= 1                                                        */
+  int32_t head_dim;      /* D; must be 128                                                  */
+  int32_t max_seq;       /* S_max, cache rows per (sequence, KV head); B*Hkv*S_max < 2^31   */
+  float scale;           /* softmax scale, usually 1/sqrt(D)                                */
+  int32_t mask_mode;     /* LA_MASK_*                                                       */
+  int32_t algo;          /* LA_ALGO_*                                                       */
+} la_pbd_cfg;
+
+/* Library version as 10000*major + 100*minor + patch. */
+int32_t la_version(void);
+
+/* Static text for a status code (never NULL). */
+const char* la_status_string(la_status status);
+
+/*
+ * Bytes of device workspace la_pbd_attn / la_pbd_step need for this configuration and window
+ * length on the current device: a 256-byte header (sticky error flags) followed by the
+ * per-split partial results (running max, running sum, unnormalised fp32 output rows).
+ * Returns 0 if the configuration is invalid or unsupported.
+ */
+size_t la_pbd_workspace_bytes(const la_pbd_cfg* cfg, int32_t window_len);
+
+/*
+ * Zero the workspace header (error flags) on `stream`. Call once after allocating a workspace;
+ * the partial-result area needs no initialisation.
+ */
+la_status la_pbd_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Step a1 -- window K/V append (RK3588 card, item 1: the prefix KV is reused, the window's
+ * tokens are written after it, with no rollback of stale speculative rows).
+ * For every b, w < W, KV head h:  k_cache[b, h, P_b + w, :] = k_new[b, w, h, :]  (same for v).
+ * Bit-exact copy. Sequences with P_b < 0 or P_b + W > max_seq are skipped (la_pbd_attn then
+ * flags them). k_new/v_new must not alias the caches.
+ */
+la_status la_kv_append(const la_pbd_cfg* cfg, const void* k_new, const void* v_new,
+                       void* k_cache, void* v_cache, const int32_t* seq_lens,
+                       int32_t window_len, void* stream);
+
+/*
+ * Steps a2..a6 -- PBD window attention over the cache (window rows already appended).
+ * q, out: bf16 [B, W, Hq, D]; caches bf16 [B, Hkv, S_max, D]; seq_lens int32 [B] on the
+ * device; 1 <= window_len <= 16. `workspace` must hold la_pbd_workspace_bytes(cfg, W) bytes
+ * whose header was zeroed once by la_pbd_workspace_init. out may not alias any input.
+ */
+la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, int32_t window_len,
+                      void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One whole layer call: la_kv_append followed by la_pbd_attn on the same stream.
+ */
+la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new,
+                      const void* v_new, void* k_cache, void* v_cache,
+                      const int32_t* seq_lens, int32_t window_len, void* out,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, read and clear the workspace's sticky device-side error flags.
+ * Returns LA_OK, LA_ERR_SEQ_OVERFLOW, LA_ERR_TIMEOUT or LA_ERR_CUDA.
+ */
+la_status la_pbd_check(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_PBD_H_ */

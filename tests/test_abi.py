@@ -1,0 +1,100 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol, and its host-side
+validation rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_masked_window_b200 as bmw
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "la_pbd.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(la_[a-z_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_masked_window_b200 import build
+    build.build()
+    return bmw.load()
+
+
+def test_header_declares_binding_symbols():
+    assert declared_functions() == sorted(bmw.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings(lib):
+    assert bmw.la_version() == 100
+    for code in range(7):
+        s = bmw.la_status_string(code)
+        assert isinstance(s, str) and s
+    assert bmw.la_status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    base = dict(batch=1, num_q_heads=16, num_kv_heads=2, max_seq=128)
+    base.update(kw)
+    return bmw.Config.make(**base)
+
+
+@pytest.mark.parametrize("kw,W,expect", [
+    (dict(), 0, 1),                        # window 0
+    (dict(), 17, 1),                       # window > 16
+    (dict(batch=0), 6, 1),
+    (dict(batch=5000), 6, 1),
+    (dict(head_dim=64), 6, 2),
+    (dict(num_q_heads=15), 6, 2),          # Hq % Hkv != 0
+    (dict(num_kv_heads=1), 16, 2),         # W * G = 256 > 128
+    (dict(mask_mode=7), 6, 1),
+    (dict(algo=9), 6, 1),
+    (dict(algo=1, num_kv_heads=1), 5, 2),  # tensor-core kernel needs W * G <= 64
+    (dict(max_seq=0), 6, 1),
+    (dict(batch=4096, num_kv_heads=16, num_q_heads=16, max_seq=1 << 20), 6, 2),
+])
+def test_host_validation(lib, kw, W, expect):
+    cfg = _cfg(**kw)
+    st = lib.la_pbd_attn(ctypes.byref(cfg), 16, 16, 16, 16, W, 16, 256, 1 << 30, None)
+    assert st == expect
+    assert bmw.la_pbd_workspace_bytes(cfg, W) == 0
+
+
+def test_null_and_misaligned_pointers(lib):
+    cfg = _cfg()
+    # null q
+    assert lib.la_pbd_attn(ctypes.byref(cfg), 0, 16, 16, 16, 6, 16, 256, 1 << 30, None) == 1
+    # misaligned k_cache (not 16-byte aligned)
+    assert lib.la_pbd_attn(ctypes.byref(cfg), 16, 24, 16, 16, 6, 16, 256, 1 << 30, None) == 1
+    # misaligned seq_lens
+    assert lib.la_pbd_attn(ctypes.byref(cfg), 16, 16, 16, 18, 6, 16, 256, 1 << 30, None) == 1
+    assert lib.la_kv_append(ctypes.byref(cfg), 0, 16, 16, 16, 16, 6, None) == 1
+    assert lib.la_kv_append(ctypes.byref(cfg), 16, 16, 16, 16, 16, 0, None) == 1
+    assert lib.la_pbd_step(ctypes.byref(cfg), 16, 16, 16, 16, 16, 16, 6, 0, 256, 1 << 30, None) == 1
+    # null config
+    assert lib.la_pbd_attn(None, 16, 16, 16, 16, 6, 16, 256, 1 << 30, None) == 1
+    # workspace checks that need no device
+    assert lib.la_pbd_workspace_init(0, 1 << 20, None) == 3
+    assert lib.la_pbd_workspace_init(256, 16, None) == 3
+    assert lib.la_pbd_check(0, None) == 3
+    assert lib.la_pbd_check(100, None) == 3
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    cfg = _cfg(max_seq=8)
+    q = torch.zeros(1, 6, 16, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        bmw.la_kv_append(cfg, q[:, :, :2], q[:, :, :2], torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16),
+                         torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16),
+                         torch.zeros(1, dtype=torch.int32), 6)

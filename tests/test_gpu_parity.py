@@ -1,0 +1,185 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Covers the five synthetic workloads at their full shapes (the multi-layer workloads on a
+subset of layers, each layer being an independent call of the same kernels), both kernels
+(tcgen05 and CUDA cores), the causal-window mask, and edge cases: empty prefix, tiny and
+ragged prefixes, window lengths 1..16, GQA group sizes, stale rows poisoned with NaN,
+invalid prefix lengths, many short sequences per CTA, and bit-exact window append.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_masked_window_b200 as bmw
+import oracle
+import workloads
+from gpu_util import assert_parity, oracle_step, run_step, to_dev
+
+pytestmark = pytest.mark.gpu
+
+ALGOS = [bmw.LA_ALGO_TCGEN05, bmw.LA_ALGO_SIMT]
+ALGO_IDS = ["tcgen05", "simt"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_lib):
+    return cuda_lib
+
+
+def _workload_case(name, layers):
+    wl = workloads.WORKLOADS[name]
+    wi = workloads.generate(wl, layers=max(layers) + 1)
+    return wl, wi
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+@pytest.mark.parametrize("name,layers", [
+    ("tiny", [0]),
+    ("single_image", [0, 17, 35]),
+    ("max_context", [0, 35]),
+    ("max_context_w1", [0, 35]),
+    ("ragged", [0]),
+    ("long", [0]),
+])
+def test_workload_parity(name, layers, algo):
+    wl, wi = _workload_case(name, layers)
+    for layer in layers:
+        li = wi.layers[layer]
+        gpu = run_step(li, wi.seq_lens, wi.max_seq, wl.window, algo=algo)
+        ref = oracle_step(li, wi.seq_lens, wl.scale)
+        assert_parity(gpu, ref, f"{name} layer {layer}")
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+@pytest.mark.parametrize("prefixes,W", [
+    ((0,), 6), ((1,), 6), ((5,), 6), ((63,), 6), ((64,), 6), ((65,), 6), ((57,), 6),
+    ((0,), 1), ((1,), 1), ((200,), 1),
+    ((10,), 2), ((77,), 3), ((129,), 4), ((300,), 5), ((31,), 7), ((1000,), 8),
+    ((0, 1, 2, 3, 4, 130, 64, 65), 6),
+])
+def test_small_prefixes(prefixes, W, algo):
+    wi = workloads.random_case(len(prefixes), prefixes, W, seed=100 + W + len(prefixes))
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, W, algo=algo)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(gpu, ref, f"P={prefixes} W={W}")
+
+
+@pytest.mark.parametrize("W", [9, 12, 16])
+def test_long_windows_simt(W):
+    wi = workloads.random_case(2, (40, 333), W, seed=7 + W)
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, W, algo=bmw.LA_ALGO_AUTO)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(gpu, ref, f"W={W}")
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+@pytest.mark.parametrize("Hq,Hkv,W", [(16, 16, 3), (8, 1, 6), (32, 4, 2), (4, 2, 6)])
+def test_gqa_groupings(Hq, Hkv, W, algo):
+    wi = workloads.random_case(2, (90, 17), W, num_q_heads=Hq, num_kv_heads=Hkv, seed=3 + Hq)
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, W, algo=algo, Hq=Hq, Hkv=Hkv)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(gpu, ref, f"Hq={Hq} Hkv={Hkv}")
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+def test_causal_window_mode(algo):
+    wi = workloads.random_case(3, (0, 70, 1500), 6, seed=41)
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=algo, mask_mode=bmw.LA_MASK_CAUSAL_WINDOW)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale, mask="causal")
+    assert_parity(gpu, ref, "causal window")
+    # and it differs from the bidirectional window
+    ref_pbd = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert np.abs(ref_pbd - ref).max() > 1e-2
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+def test_stale_rows_never_read(algo):
+    """Cache rows at and beyond P + W hold NaN: they must not reach the output."""
+    wi = workloads.random_case(3, (7, 64, 250), 6, seed=5, max_seq=400, stale_fill=float("nan"))
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=algo)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(gpu, ref, "stale NaN rows")
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+def test_many_short_sequences(algo):
+    """Hundreds of short sequences: CTAs own many whole sequences plus split ones."""
+    rng = np.random.default_rng(9)
+    prefixes = tuple(int(x) for x in rng.integers(0, 90, size=300))
+    wi = workloads.random_case(300, prefixes, 6, num_q_heads=16, num_kv_heads=2, seed=9)
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=algo)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(gpu, ref, "300 short sequences")
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+def test_invalid_prefix_lengths_flagged(algo):
+    """P < 0 or P + W > max_seq: zero output rows, untouched cache, sticky status."""
+    wi = workloads.random_case(4, (10, 20, 30, 40), 6, seed=13, max_seq=64)
+    li = wi.layers[0]
+    bad = wi.seq_lens.clone()
+    bad[1] = -3
+    bad[2] = 60           # 60 + 6 > 64
+    out, kc, vc, ws = run_step(li, bad, wi.max_seq, 6, algo=algo, return_cache=True)
+    assert bmw.la_pbd_check(ws) == 5
+    assert bmw.la_pbd_check(ws) == 0   # cleared by the first read
+    assert torch.equal(out[1], torch.zeros_like(out[1]))
+    assert torch.equal(out[2], torch.zeros_like(out[2]))
+    assert torch.equal(kc[1], li.k_cache[1]) and torch.equal(vc[2], li.v_cache[2])
+    good = [0, 3]
+    sub = workloads.LayerInputs(li.q[good], li.k_cache[good], li.v_cache[good], li.k_new[good],
+                                li.v_new[good])
+    ref = oracle_step(sub, wi.seq_lens[good], wi.workload.scale)
+    assert_parity(out[good], ref, "valid sequences beside invalid ones")
+
+
+def test_kv_append_bit_exact():
+    wi = workloads.random_case(5, (0, 3, 64, 100, 250), 6, seed=17, max_seq=300)
+    li = wi.layers[0]
+    cfg = bmw.Config.make(5, 16, 2, wi.max_seq)
+    kc, vc = to_dev(li.k_cache), to_dev(li.v_cache)
+    bmw.la_kv_append(cfg, to_dev(li.k_new), to_dev(li.v_new), kc, vc, to_dev(wi.seq_lens), 6)
+    torch.cuda.synchronize()
+    k_ref, v_ref = oracle.kv_append(li.k_cache, li.v_cache, li.k_new, li.v_new, wi.seq_lens)
+    assert np.array_equal(kc.cpu().double().numpy(), k_ref)
+    assert np.array_equal(vc.cpu().double().numpy(), v_ref)
+
+
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+def test_deterministic_and_no_stray_writes(algo):
+    wi = workloads.random_case(2, (500, 1200), 6, seed=21)
+    li = wi.layers[0]
+    cfg = bmw.Config.make(2, 16, 2, wi.max_seq, algo=algo)
+    q = to_dev(li.q)
+    kc, vc = to_dev(li.k_cache), to_dev(li.v_cache)
+    sl = to_dev(wi.seq_lens)
+    bmw.la_kv_append(cfg, to_dev(li.k_new), to_dev(li.v_new), kc, vc, sl, 6)
+    guard = torch.full((3 * q.numel() + 2 * 4096,), 12345.0).to(torch.bfloat16).cuda()
+    lo = 4096 + q.numel()
+    out = guard[lo:lo + q.numel()].view_as(q)
+    ws = bmw.Workspace(cfg, 6)
+    bmw.la_pbd_attn(cfg, q, kc, vc, sl, 6, out, ws)
+    first = out.clone()
+    bmw.la_pbd_attn(cfg, q, kc, vc, sl, 6, out, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(first, out)
+    g = guard.cpu()
+    assert (g[:lo] == g[0]).all()
+    assert (g[lo + q.numel():] == g[0]).all()
+    assert bmw.la_pbd_check(ws) == 0
+
+
+def test_kernels_agree():
+    """tcgen05 and CUDA-core kernels on the same inputs agree to rounding."""
+    wi = workloads.random_case(4, (100, 2000, 4096, 31), 6, seed=33)
+    li = wi.layers[0]
+    a = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=bmw.LA_ALGO_TCGEN05).double()
+    b = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=bmw.LA_ALGO_SIMT).double()
+    rel = float((a - b).norm() / b.norm())
+    assert rel < 2e-3, rel
