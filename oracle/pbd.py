@@ -166,16 +166,21 @@ def window_attention(q, k_cache, v_cache, seq_lens, scale: float,
             M = causal_window_mask(int(P[b]), W, S)
         else:
             raise ValueError(mask)
+        # The sums run over keys some window row may see, j < T; rows at or beyond T are
+        # never part of the definition (their content may be anything, even non-finite).
+        cols = np.nonzero(M.any(axis=0))[0]
+        T = int(cols.max()) + 1 if cols.size else 0
+        Mt = M[:, :T]
         for h in range(Hq):
             g = kv_head_of(h, Hq, Hkv)
-            s = scale * (qf[b, :, h, :] @ kf[b, g, :, :].T)          # [W, S]
-            s = np.where(M, s, -np.inf)
+            s = scale * (qf[b, :, h, :] @ kf[b, g, :T, :].T)          # [W, T]
+            s = np.where(Mt, s, -np.inf)
             s = s - s.max(axis=1, keepdims=True)
-            e = np.where(M, np.exp(s), 0.0)
+            e = np.where(Mt, np.exp(s), 0.0)
             p = e / e.sum(axis=1, keepdims=True)
-            out[b, :, h, :] = p @ vf[b, g, :, :]
+            out[b, :, h, :] = p @ vf[b, g, :T, :]
             if return_probs:
-                probs[b, h] = p
+                probs[b, h, :, :T] = p
     if return_probs:
         return out, probs
     return out

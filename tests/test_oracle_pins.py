@@ -314,6 +314,6 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     for pin in PINS:
         try:
             pin(opbd)
-        except AssertionError:
+        except Exception:  # an assertion, or the broken oracle failing outright
             failures += 1
     assert failures > 0, f"no pin caught the planted mistake {name!r}"
