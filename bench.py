@@ -179,7 +179,7 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
     clk = clocks.stop()
     ms = max_over_ranks(ms)
     ms_per_step = ms / steps
-    value = world * B * steps / (ms / 1e3)
+    value = aggregate_throughput(world, B, steps, ms)
 
     # Dominant kernel: the attention call of one layer (attention + split merge), timed alone
     # over the same rotating copies.
@@ -222,7 +222,7 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
         torch.cuda.synchronize()
         barrier()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": world * B * steps / (ms_e2e / 1e3), "unit": UNIT,
+        e2e = {"value": aggregate_throughput(world, B, steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ms_e2e / steps}
     del step_graphs, attn_graphs
@@ -232,6 +232,30 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
         "step_bytes": step_bytes, "copies": copies, "e2e": e2e, "layers": L,
         "launches_per_step": L * 3,
     }
+
+
+def dist_helpers(world, device):
+    """Barrier and max-over-ranks reduction for the timing (the only collective used: the
+    replicas share no data)."""
+    if world <= 1:
+        return (lambda: None), (lambda x: x)
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        dist.barrier()
+
+    def max_over_ranks(x):
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return barrier, max_over_ranks
+
+
+def aggregate_throughput(world, batch, steps, max_ms):
+    """Whole-job window-steps/s: every replica runs `batch` sequences for `steps` steps; the
+    job takes as long as its slowest rank."""
+    return world * batch * steps / (max_ms / 1e3)
 
 
 def cpu_baseline(wl, budget_s):
@@ -277,6 +301,7 @@ def main():
                     help="extra workloads measured for the prefix-length sweep ('' for none)")
     ap.add_argument("--max-copies", type=int, default=16)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -309,19 +334,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         device = torch.device("cuda", local_rank)
-
-        def barrier():
-            dist.barrier()
-
-        def max_over_ranks(x):
-            t = torch.tensor([x], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
     else:
         device = torch.device("cuda", 0)
         torch.cuda.set_device(0)
-        barrier = lambda: None  # noqa: E731
-        max_over_ranks = lambda x: x  # noqa: E731
+    barrier, max_over_ranks = dist_helpers(world, device)
 
     res = measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks)
     peak, peak_kind = measured_peaks()
@@ -346,7 +362,7 @@ def main():
             import torch.distributed as dist
             dist.destroy_process_group()
         return
-    cb = cpu_baseline(wl, args.cpu_budget) if world == 1 else None
+    cb = cpu_baseline(wl, args.cpu_budget) if (world == 1 and not args.no_cpu) else None
     wi = res["wi"]
     line = {
         "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,

@@ -6,23 +6,30 @@
 // rounded to bf16 (RNE). Sequences held whole by one CTA were written by the attention kernel
 // and are skipped here. Sequences with an invalid prefix length (no visible keys) get zero
 // rows and raise the sticky overflow flag.
+//
+// One warp per output row (4 rows per 128-thread block): lanes first reduce the row's
+// maxima and sums over the partials, keeping the weights in shared memory, then each lane
+// accumulates 4 of the 128 channels over the partials with independent 16-byte loads.
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 
 namespace la {
 
-__global__ void __launch_bounds__(256) pbd_combine_kernel(Problem p) {
-  const int s = blockIdx.x;            // sequence = b * Hkv + h
+constexpr int kCombineRows = 4;
+constexpr int kCombineMaxSlots = 1024;   // >= partials of one sequence (<= grid size)
+
+__global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem p) {
+  __shared__ float s_w[kCombineRows][kCombineMaxSlots];
+  const int s = blockIdx.y;            // sequence = b * Hkv + h
   const int b = s / p.Hkv, h = s - b * p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kCombineRows + warp;
   const int n = p.pre_g[b + 1] - p.pre_g[b];
-  const int nthr = blockDim.x;
+  if (r >= p.R) return;
+  __nv_bfloat16* dst = p.out + out_row_offset(p, b, h, r);
   if (n == 0) {
-    for (int idx = threadIdx.x; idx < p.R * (kHeadDim / 8); idx += nthr) {
-      int r = idx / (kHeadDim / 8), c = idx % (kHeadDim / 8);
-      *reinterpret_cast<uint4*>(p.out + out_row_offset(p, b, h, r) + c * 8) =
-          make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (threadIdx.x == 0 && h == 0) atomicOr(&p.hdr->err, kErrSeqOverflow);
+    reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
+    if (lane == 0 && r == 0 && h == 0) atomicOr(&p.hdr->err, kErrSeqOverflow);
     return;
   }
   const long long T = (long long)p.Hkv * p.pre_g[p.B];
@@ -30,38 +37,62 @@ __global__ void __launch_bounds__(256) pbd_combine_kernel(Problem p) {
   const long long off = (long long)p.Hkv * p.pre_g[b] + (long long)h * n;
   const int c0 = (int)(off / C), c1 = (int)((off + n - 1) / C);
   if (c0 == c1) return;
+  const int ns = c1 - c0 + 1;
+  const size_t stride = slot_floats(p.rows_pad);
+  const float* base = p.partials + (size_t)(c0 + s) * stride;
 
-  // One thread per (row, 4 channels).
-  for (int idx = threadIdx.x; idx < p.R * (kHeadDim / 4); idx += nthr) {
-    const int r = idx / (kHeadDim / 4), d = (idx % (kHeadDim / 4)) * 4;
-    float M = -INFINITY;
-    for (int c = c0; c <= c1; ++c) M = fmaxf(M, slot_ptr(p, c + s)[r]);
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = c0; c <= c1; ++c) {
-      const float* sl = slot_ptr(p, c + s);
-      const float mk = sl[r];
-      if (mk == -INFINITY) continue;
-      const float w = fast_exp2(mk - M);
-      L = fmaf(w, sl[p.rows_pad + r], L);
-      const float4 a = *reinterpret_cast<const float4*>(sl + 2 * p.rows_pad + (size_t)r * kHeadDim + d);
-      acc.x = fmaf(w, a.x, acc.x);
-      acc.y = fmaf(w, a.y, acc.y);
-      acc.z = fmaf(w, a.z, acc.z);
-      acc.w = fmaf(w, a.w, acc.w);
-    }
-    const float inv = 1.f / L;
-    __nv_bfloat162 o01 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    __nv_bfloat162 o23 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t*>(&o01);
-    packed.y = *reinterpret_cast<uint32_t*>(&o23);
-    *reinterpret_cast<uint2*>(p.out + out_row_offset(p, b, h, r) + d) = packed;
+  float M = -INFINITY;
+  for (int k = lane; k < ns; k += 32) M = fmaxf(M, base[k * stride + r]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  for (int k = lane; k < ns; k += 32) {
+    const float mk = base[k * stride + r];
+    const float w = (mk == -INFINITY) ? 0.f : fast_exp2(mk - M);
+    s_w[warp][k] = w;
+    L = fmaf(w, base[k * stride + p.rows_pad + r], L);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  __syncwarp();
+
+  const float* acc0 = base + 2 * p.rows_pad + (size_t)r * kHeadDim + 4 * lane;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int k = 0;
+  for (; k + 4 <= ns; k += 4) {
+    float4 a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = *reinterpret_cast<const float4*>(acc0 + (size_t)(k + u) * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float w = s_w[warp][k + u];
+      acc.x = fmaf(w, a[u].x, acc.x);
+      acc.y = fmaf(w, a[u].y, acc.y);
+      acc.z = fmaf(w, a[u].z, acc.z);
+      acc.w = fmaf(w, a[u].w, acc.w);
+    }
+  }
+  for (; k < ns; ++k) {
+    const float4 a = *reinterpret_cast<const float4*>(acc0 + (size_t)k * stride);
+    const float w = s_w[warp][k];
+    acc.x = fmaf(w, a.x, acc.x);
+    acc.y = fmaf(w, a.y, acc.y);
+    acc.z = fmaf(w, a.z, acc.z);
+    acc.w = fmaf(w, a.w, acc.w);
+  }
+  const float inv = 1.f / L;
+  __nv_bfloat162 o01 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  __nv_bfloat162 o23 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 packed;
+  packed.x = *reinterpret_cast<uint32_t*>(&o01);
+  packed.y = *reinterpret_cast<uint32_t*>(&o23);
+  reinterpret_cast<uint2*>(dst)[lane] = packed;
 }
 
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream) {
-  pbd_combine_kernel<<<p.B * p.Hkv, 256, 0, stream>>>(p);
+  if (p.num_ctas > kCombineMaxSlots) return cudaErrorInvalidValue;
+  dim3 grid((p.R + kCombineRows - 1) / kCombineRows, p.B * p.Hkv);
+  pbd_combine_kernel<<<grid, 32 * kCombineRows, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

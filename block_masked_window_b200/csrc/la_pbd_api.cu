@@ -53,6 +53,7 @@ la_status check_cfg(const la_pbd_cfg* cfg, int32_t W) {
   // Per-head prefix sums and TMA row coordinates are int32: B * Hkv * S_max < 2^31.
   if ((long long)cfg->batch * cfg->num_kv_heads * cfg->max_seq >= (1LL << 31))
     return LA_ERR_UNSUPPORTED;
+  if ((long long)cfg->batch * cfg->num_kv_heads > 65535) return LA_ERR_UNSUPPORTED;
   const long long R = (long long)W * (cfg->num_q_heads / cfg->num_kv_heads);
   if (R > 128) return LA_ERR_UNSUPPORTED;
   if (cfg->algo == LA_ALGO_TCGEN05 && R > 64) return LA_ERR_UNSUPPORTED;
@@ -82,6 +83,14 @@ la_status fill_problem(const la_pbd_cfg* cfg, int32_t W, Problem* p) {
   p->mask_mode = cfg->mask_mode;
   p->scale_log2 = cfg->scale * 1.4426950408889634f;
   return LA_OK;
+}
+
+// Grid size: the resident capacity, but no more CTAs than the largest possible key stream
+// (every sequence at full capacity) can keep busy at c_min keys each.
+int grid_for(const Problem& p, int capacity) {
+  const long long max_tokens = (long long)p.B * p.Hkv * p.S;
+  const long long useful = (max_tokens + p.c_min - 1) / p.c_min;
+  return (int)(useful < capacity ? (useful < 1 ? 1 : useful) : capacity);
 }
 
 }  // namespace
@@ -175,8 +184,8 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
   if (algo == LA_ALGO_TCGEN05) {
     la::TmaMaps maps;
     if (la::make_tma_maps(p, &maps) != cudaSuccess) return LA_ERR_CUDA;
-    p.num_ctas = sms * la::tc_ctas_per_sm();
     p.c_min = la::tc_min_chunk();
+    p.num_ctas = grid_for(p, sms * la::tc_ctas_per_sm());
     e = la::launch_attn_tc(p, &maps.k, &maps.v, &maps.q, s);
   } else {
     int per_sm = 0;
@@ -184,8 +193,8 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
     if (e != cudaSuccess) return LA_ERR_CUDA;
     if (per_sm < 1) return LA_ERR_UNSUPPORTED;
     if (per_sm > la::kMaxCtasPerSm) per_sm = la::kMaxCtasPerSm;
-    p.num_ctas = sms * per_sm;
     p.c_min = 32;
+    p.num_ctas = grid_for(p, sms * per_sm);
     e = la::launch_attn_simt(p, s);
   }
   if (e != cudaSuccess) return LA_ERR_CUDA;
