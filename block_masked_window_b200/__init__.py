@@ -16,7 +16,7 @@ __all__ = [
     "LA_MASK_PBD", "LA_MASK_CAUSAL_WINDOW", "LA_ALGO_AUTO", "LA_ALGO_TCGEN05", "LA_ALGO_SIMT",
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
-    "la_pbd_step", "la_pbd_check", "Workspace", "EXPORTED_SYMBOLS",
+    "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "Workspace", "EXPORTED_SYMBOLS",
 ]
 
 LA_MASK_PBD = 0
@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
 
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
-                    "la_pbd_check"]
+                    "la_pbd_check", "la_pbd_attn_static"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: Optional[ctypes.CDLL] = None
@@ -92,6 +92,8 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_step.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.la_pbd_check.restype = i32
     lib.la_pbd_check.argtypes = [vp, vp]
+    lib.la_pbd_attn_static.restype = i32
+    lib.la_pbd_attn_static.argtypes = [cfgp, vp, vp, vp, vp, i32, vp, vp]
     _LIB = lib
     return lib
 
@@ -213,3 +215,23 @@ def la_pbd_step(cfg: Config, q, k_new, v_new, k_cache, v_cache, seq_lens, window
 def la_pbd_check(workspace: Workspace, stream=None) -> int:
     """Synchronise and return the sticky device status (0 = LA_OK); clears it."""
     return int(load().la_pbd_check(workspace.data_ptr(), _stream(stream)))
+
+
+def la_pbd_attn_static(cfg: Config, q, k_cache, v_cache, seq_lens, window_len: int, out,
+                       stream=None) -> None:
+    """Window attention without a caller-provided workspace.
+
+    For callers that cannot allocate device memory (an engine plugin given no scratch, a
+    loop where cudaMalloc is not allowed): the library keeps one 32 MiB scratch array per
+    GPU. Calls that overlap on the GPU share that array and race; serialise them.
+    """
+    W = int(window_len)
+    q_shape, cache_shape, _ = _shapes(cfg, W)
+    _check_tensor(q, "q", "bf16", q_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check_tensor(out, "out", "bf16", q_shape)
+    _check(load().la_pbd_attn_static(ctypes.byref(cfg), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(seq_lens), W, _ptr(out), _stream(stream)),
+           "la_pbd_attn_static")

@@ -17,7 +17,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libla_pbd.so")
-SOURCES = ["la_pbd_api.cu", "kv_append.cu", "attn_simt.cu", "attn_tc.cu", "combine.cu"]
+SOURCES = ["la_pbd_api.cu", "kv_append.cu", "attn_simt.cu", "attn_tc.cu", "combine.cu",
+           "la_pbd_static.cu"]
 
 
 def nvcc() -> str:

@@ -131,6 +131,27 @@ la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new,
                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * la_pbd_attn without a caller-provided workspace, for callers that cannot allocate device
+ * memory: a plugin inside a host engine that owns all device memory and offers its kernels no
+ * scratch, or a latency-critical loop in which cudaMalloc is not allowed because it can
+ * synchronise the device and take an unbounded time. The paper has no counterpart; this is a
+ * deployment convenience of this library.
+ * Runs the same kernels as la_pbd_attn with their scratch in one file-scope device array of
+ * 32 MiB that every GPU loading the library holds until the process exits; the call itself
+ * allocates and frees nothing. Configurations whose la_pbd_workspace_bytes exceeds 32 MiB are
+ * rejected with LA_ERR_WORKSPACE (nothing enqueued). The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. All calls on a device share the one array and it keeps the last
+ * call's contents: calls whose executions overlap on the GPU (other streams, concurrent
+ * threads) race on it and must be serialised by the caller. Device-side per-sequence errors
+ * still produce zero rows, but their sticky flag stays in the shared array and is not readable
+ * through la_pbd_check.
+ */
+la_status la_pbd_attn_static(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* seq_lens, int32_t window_len,
+                             void* out, void* stream);
+
+/*
  * Synchronise `stream`, read and clear the workspace's sticky device-side error flags.
  * Returns LA_OK, LA_ERR_SEQ_OVERFLOW, LA_ERR_TIMEOUT or LA_ERR_CUDA.
  */
