@@ -3,30 +3,42 @@
 // Steps a2..a5 of one PBD decode step (LocateAnything-3B for RK3588 model card, "How it
 // differs from the original", item 1: the window attends bidirectionally to itself and
 // causally to the prefix, so every window row sees keys [0, P_b + W)). The R = W * G query
-// rows that share one KV head (window row i, grouped head g -> row i*G + g; G = Hq / Hkv) form
-// the M = 64 side of two tensor-core products per 64-key tile:
-//   S  = Q  K^T   (M=64 rows, N=64 keys,     K=128 channels)  -> TMEM, fp32
-//   O  = P  V     (M=64 rows, N=128 channels, K=64 keys)       -> TMEM, fp32
-// P is the online-softmax probability tile. To keep fp32-level accuracy through a bf16
-// tensor-core product, P is split as P = P_hi + P_lo with both halves bf16 (error ~2^-17 P)
-// and O takes two MMAs per k-step; the tensor core has ample headroom at this arithmetic
-// intensity (48 flop per byte of K/V at W = 6), so the path stays bound by HBM.
+// rows that share one KV head (window row i, grouped head g -> row q = i*G + g) are the
+// narrow N side of two tensor-core products per 128-key tile, and the keys (or channels) are
+// the full-rate M = 128 side:
+//   S^T = K  Q^T   (M = 128 keys,     N = NQ rows,       K = 128 channels) -> TMEM fp32
+//   O^T = V^T P^T  (M = 128 channels, N = 2 NQ (hi, lo), K = 128 keys)     -> TMEM fp32
+//   L   = 1   P^T  (M = 128 copies,   N = 2 NQ (hi, lo), K = 128 keys)     -> TMEM fp32
+// The last product, against a constant all-ones tile, accumulates the softmax row sums next
+// to O, so rescaling, precision and the final normalisation treat O and l identically and no
+// thread has to keep or reduce partial sums.
+// NQ = R rounded up to 16 (48 for the PBD window of 6 rows x 8 grouped heads). P is split
+// into P_hi + P_lo (both bf16, residual ~2^-17 P) so that the bf16 tensor-core product keeps
+// fp32-level accuracy; both halves ride in one N = 2 NQ MMA that reads the V tile once.
 //
-// Roles (192 threads, 2 CTAs per SM, 256 TMEM columns each):
-//   warp 0      TMA producer: Q once per segment, K/V tiles into a 2-stage ring
-//   warp 1      TMEM owner and single-thread MMA issuer
-//   warps 2..5  softmax / accumulation: warp w reads TMEM sub-partition w % 4, i.e. rows
-//               16*(w%4) .. +15 of the 64-row accumulators, through 16x256b loads whose
-//               per-thread layout is (row t/4 and t/4+8, columns 2*(t%4) + {0,1} per 8)
-// The softmax warps keep the running output in registers: every PV product lands in a fresh
-// TMEM tile that they fold in as O <- alpha * O + PV, so no TMEM read-modify-write is needed.
+// Online softmax with a lazy reference maximum: per row q the kernel keeps a reference m_q
+// (log2 domain) and uses p = 2^(x - m_q). The reference is raised (and O, l rescaled) only
+// when some score of a tile exceeds it by more than 2^8, which a CTA-wide vote detects
+// without reducing across keys; the full cross-key maximum is computed only then (always on a
+// segment's first tile). O accumulates in TMEM over the whole segment, so a tile without a
+// rescale touches O only through the MMA.
 //
-// Shared-memory tiles use the 128-byte swizzle written by TMA, which is also the canonical
-// SWIZZLE_128B operand layout of the tensor core: K-major for Q, K and P, MN-major for V.
+// Roles (224 threads, 1 CTA per SM):
+//   warp 0      TMA producer of Q (once per segment, double-buffered) and the K ring
+//   warp 6      TMA producer of the V ring (so neither ring waits on the other)
+//   warp 1      TMEM owner and single-thread MMA issuer (non-blocking: issues whichever of
+//               the next S^T or the next O^T product is ready first)
+//   warps 2..5  softmax: thread t of the 128 reads TMEM lane t, i.e. key t of the S^T tile
+//               and channel t of the O^T accumulator
 //
-// Every mbarrier wait is bounded: after ~2 s of waiting the CTA raises the sticky timeout
-// flag in the workspace header, the other roles stop at their next wait, in-flight copies
-// and MMAs are drained with bounded waits, TMEM is freed and the kernel returns.
+// Shared-memory operand layouts: K, V and Q use the 128-byte swizzle written by TMA (K-major
+// for K and Q, MN-major for V as the A operand of O^T); P^T is written by the softmax
+// threads as an MN-major, non-swizzled operand (8x8 core matrices: rows of 16 bytes, key
+// groups 128 bytes apart, row groups 2048 bytes apart), one 16-byte store per 8 rows.
+//
+// Every mbarrier wait is bounded: after ~2 s the CTA raises the sticky timeout flag in the
+// workspace header, the other roles stop at their next wait, in-flight copies and MMAs are
+// drained with bounded waits, TMEM is freed and the kernel returns.
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 #include "tma_util.h"
@@ -34,52 +46,77 @@
 namespace la {
 namespace {
 
-constexpr int kNT = kTileKeys;         // keys per tile
-constexpr int kStages = 2;
-constexpr int kThreadsTc = 192;
-constexpr int kTmemCols = 256;
-constexpr int kColO = 128;             // O accumulator columns [128, 256); S buffers at 0, 64
+constexpr int kNT = kTileKeys;          // 128 keys per tile
+constexpr int kKStages = 2;
+constexpr int kSBufs = 4;               // S^T buffers in TMEM: QK may run kSBufs-1 tiles ahead
+constexpr int kThreadsTc = 224;
+constexpr int kTmemCols = 512;
+constexpr int kHalfBytes = kNT * 128;   // 128 rows x 128 B: one swizzle column of a K/V tile
+constexpr int kTileBytes = 2 * kHalfBytes;
+constexpr float kLazyThreshold = 8.f;   // log2 units: p stays <= 2^8 between rescales
+constexpr long long kWaitLimitNs = 2000000000LL;
+constexpr int kNamedBarSoftmax = 1;
 
-constexpr int kHalfBytes = 64 * 128;            // 64 rows x 128 B (one swizzle column)
-constexpr int kQBytes = 2 * kHalfBytes;         // Q: 2 halves of 64 channels
-constexpr int kTileBytes = 2 * kHalfBytes;      // one K (or V) tile: 2 halves
-constexpr int kStageBytes = 2 * kTileBytes;     // K + V
-constexpr int kOffQ = 0;
-constexpr int kOffStage = kOffQ + kQBytes;
-constexpr int kOffPhi = kOffStage + kStages * kStageBytes;
-constexpr int kOffPlo = kOffPhi + kHalfBytes;
-constexpr int kOffBar = kOffPlo + kHalfBytes;
-constexpr int kNumBars = 16;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag
-constexpr int kOffPre = kOffMisc + 64;
+// Barrier indices (K ring, V ring sized at run time up to kMaxVStages). Every barrier is waited
+// with a phase parity, which is only sound if its producer can never complete two phases
+// ahead of a waiter. Each ring below is sized so that refilling a slot requires its previous
+// consumer to have finished: e.g. the softmax can only refill a P^T buffer after the PV
+// product that read it completed, so P-full is per buffer (a single P-full barrier could be
+// lapped while the MMA issuer is busy).
+constexpr int kMaxVStages = 3;
+constexpr int kBarKFull = 0;
+constexpr int kBarKEmpty = kBarKFull + kKStages;
+constexpr int kBarVFull = kBarKEmpty + kKStages;
+constexpr int kBarVEmpty = kBarVFull + kMaxVStages;
+constexpr int kBarQFull = kBarVEmpty + kMaxVStages;   // [2]: Q is double-buffered
+constexpr int kBarQEmpty = kBarQFull + 2;            // [2]
+constexpr int kBarSFull = kBarQEmpty + 2;            // [kSBufs]
+constexpr int kBarPFull = kBarSFull + kSBufs;            // [2]: one per P^T buffer
+constexpr int kBarOFull = kBarPFull + 2;            // [2]: one per P^T buffer
+constexpr int kBarDrain = kBarOFull + 2;
+constexpr int kNumBars = kBarDrain + 1;
 
-// Barrier indices.
-constexpr int kBarFull = 0;     // [kStages]
-constexpr int kBarEmpty = 2;    // [kStages]
-constexpr int kBarQFull = 4;
-constexpr int kBarQEmpty = 5;
-constexpr int kBarSFull = 6;    // [2]
-constexpr int kBarPFull = 8;
-constexpr int kBarOFull = 9;
-constexpr int kBarDrain = 10;
-
-constexpr long long kWaitLimitNs = 2000000000LL;   // 2 s
-
-// Instruction descriptors (kind::f16): D fp32 (bit 4), A bf16 (bits 7..9 = 1),
-// B bf16 (bits 10..12 = 1), B major bit 16, N >> 3 at bit 17, M >> 4 at bit 24.
-constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kNT >> 3) << 17) |
-                              ((uint32_t)(64 >> 4) << 24);
-constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                              ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
+// Shared-memory plan for a given NQ and V ring depth.
+struct TcLayout {
+  int k, v, q, p, ones, bar, misc, vote, wmax, lim, mref, pre, end;
+};
+__host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, int B) {
+  // Operand buffers are 1024-byte multiples from a 1024-aligned base; every small region is
+  // rounded to 16 bytes (the per-row references are read as float4).
+  auto a16 = [](int x) { return (x + 15) & ~15; };
+  TcLayout L;
+  L.k = 0;
+  L.v = L.k + kKStages * kTileBytes;
+  L.q = L.v + vstages * kTileBytes;
+  L.p = L.q + qbufs * 2 * nq * 128;         // Q: qbufs buffers x two 64-channel halves
+  L.ones = L.p + 2 * nq * 512;              // P^T: 2 buffers x 2*nq/8 row groups of 2048 B
+  L.bar = L.ones + 128;                     // ones: one 8x8 bf16 core matrix, read with zero strides
+  L.misc = a16(L.bar + kNumBars * 8);       // tmem slot, abort flag
+  L.vote = L.misc + 16;                     // (unused slot kept for alignment)
+  L.wmax = L.vote + 32;                     // [2][4][nq] floats
+  L.lim = a16(L.wmax + 2 * 4 * nq * 4);     // [3][nq] ints: (unused), output offsets, key limits
+  L.mref = a16(L.lim + 3 * nq * 4);         // [2][nq]: per-row references
+  L.pre = a16(L.mref + 2 * nq * 4);         // [B+1] + 32 ints
+  L.end = L.pre + (round_up(B + 1, 4) + 32) * 4;
+  return L;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// Shared-memory matrix descriptor, SWIZZLE_128B (layout type 2), descriptor version 1.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
-         ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+// Shared-memory matrix descriptor (descriptor version 1). layout: 2 = SWIZZLE_128B, 0 = none.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                          uint32_t layout) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+// Instruction descriptor, kind::f16: D fp32 (bit 4), A and B bf16 (bits 7, 10),
+// A major bit 15, B major bit 16 (1 = MN-major), N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
 __device__ __forceinline__ long long now_ns() {
@@ -87,7 +124,6 @@ __device__ __forceinline__ long long now_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
 }
@@ -110,6 +146,19 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase completion (never suspends the thread).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 struct Ctl {
   volatile int* abort_flag;
   WsHeader* hdr;
@@ -117,14 +166,13 @@ struct Ctl {
 
 // Bounded wait for the completion of phase `parity`. Returns false when the CTA is aborting.
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& ctl) {
-  const long long limit_ns = kWaitLimitNs;
   if (mbar_try(bar, parity)) return true;
   const long long t0 = now_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*ctl.abort_flag) return false;
-      if (now_ns() - t0 > limit_ns) {
+      if (now_ns() - t0 > kWaitLimitNs) {
         *ctl.abort_flag = 1;
         atomicOr(&ctl.hdr->err, kErrTimeout);
         return false;
@@ -178,37 +226,58 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-
-// 16 lanes x 256 bits, repeated 8 times: 32 registers (columns 8k + 2(t%4) + {0,1}).
-__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, float (&v)[32]) {
-  uint32_t* r = reinterpret_cast<uint32_t*>(v);
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
+__device__ __forceinline__ void softmax_bar() {
+  asm volatile("bar.sync %0, 128;" ::"n"(kNamedBarSoftmax) : "memory");
 }
-// Same shape repeated 4 times: 16 registers.
-__device__ __forceinline__ void tmem_ld_x4(uint32_t taddr, float (&v)[16]) {
+
+// 32 lanes x 32 bits, 16 consecutive columns: thread i gets lane (base + i), 16 registers.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
   asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 
-__device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat162 v) {
+// OR of a predicate over the 128 softmax threads (named barrier 1), returned to all of them.
+__device__ __forceinline__ bool softmax_bar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kNamedBarSoftmax)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ float warp_max_f32(float x) {
+  float r;
+  asm volatile("redux.sync.max.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
@@ -216,37 +285,61 @@ __device__ __forceinline__ int tiles_of(const Segment& sg) { return (sg.j1 - sg.
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreadsTc, 2)
+template <int NQ, bool CAUSAL>
+__global__ void __launch_bounds__(kThreadsTc, 1)
     pbd_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                       const __grid_constant__ CUtensorMap tmq, Problem p) {
+                       const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
+                       Problem p, int ring) {
+  static_assert(NQ % 16 == 0 && NQ >= 16 && NQ <= 64, "NQ");
+  constexpr int kQHalf = NQ * 128;                 // bytes of one 64-channel half of Q
+  constexpr int kColS = 0;                         // S^T buffers at [0, kSBufs NQ)
+  constexpr int kColO = kSBufs * NQ;               // O^T (hi | lo)
+  constexpr int kColL = (kSBufs + 2) * NQ;         // row sums (hi | lo)
+  static_assert((kSBufs + 4) * NQ <= kTmemCols, "TMEM columns");
+  constexpr uint32_t kIdescQK = idesc_f16(128, NQ, 0, 0);
+  constexpr uint32_t kIdescPV = idesc_f16(128, 2 * NQ, 1, 1);
+  constexpr uint32_t kIdescL = idesc_f16(128, 2 * NQ, 0, 1);
+
   extern __shared__ __align__(1024) char smem_raw[];
   char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int vstages = ring & 0xff, qbufs = ring >> 8;   // V ring depth, Q buffers
+  const TcLayout L = tc_layout(NQ, vstages, qbufs, p.B);
   const uint32_t sb = smem_u32(base);
-  const uint32_t sQ = sb + kOffQ, sStage = sb + kOffStage, sPhi = sb + kOffPhi, sPlo = sb + kOffPlo;
-  const uint32_t sBar = sb + kOffBar;
-  auto bar = [&](int i) { return sBar + 8u * (uint32_t)i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
-  int* pre = reinterpret_cast<int*>(base + kOffPre);
+  const uint32_t sK = sb + L.k, sV = sb + L.v, sQ = sb + L.q, sP = sb + L.p, sOnes = sb + L.ones;
+  auto bar = [&](int i) { return sb + (uint32_t)L.bar + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L.misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L.misc + 8);
+  float* wmax = reinterpret_cast<float*>(base + L.wmax);
+  int* lim_s = reinterpret_cast<int*>(base + L.lim);
+  int* pre = reinterpret_cast<int*>(base + L.pre);
   int* warp_tot = pre + round_up(p.B + 1, 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Ctl ctl{abort_flag, p.hdr};
 
-  // Q padding rows R..63 must read as zero: clear the Q tile once (TMA rewrites rows < R).
-  for (int i = tid; i < kQBytes / 16; i += kThreadsTc)
-    reinterpret_cast<uint4*>(base + kOffQ)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // Q rows R..NQ-1 must read as zero: clear both Q buffers once (TMA rewrites rows < R).
+  for (int i = tid; i < 4 * kQHalf / 16; i += kThreadsTc)
+    reinterpret_cast<uint4*>(base + L.q)[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < 128 / 16; i += kThreadsTc)     // bf16 1.0 = 0x3F80
+    reinterpret_cast<uint4*>(base + L.ones)[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
     }
-    mbar_init(bar(kBarQFull), 1);
-    mbar_init(bar(kBarQEmpty), 1);
-    mbar_init(bar(kBarSFull + 0), 1);
-    mbar_init(bar(kBarSFull + 1), 1);
-    mbar_init(bar(kBarPFull), 128);
-    mbar_init(bar(kBarOFull), 1);
+    for (int s = 0; s < kMaxVStages; ++s) {
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarQFull + s), 1);
+      mbar_init(bar(kBarQEmpty + s), 1);
+    }
+    for (int s = 0; s < kSBufs; ++s) mbar_init(bar(kBarSFull + s), 1);
+    mbar_init(bar(kBarPFull + 0), 128);
+    mbar_init(bar(kBarPFull + 1), 128);
+    mbar_init(bar(kBarOFull + 0), 1);
+    mbar_init(bar(kBarOFull + 1), 1);
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -271,38 +364,63 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   const long long C = plan_chunk(p, T);
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer: Q, K
     if (lane == 0) {
       SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
       Segment sg;
       int g = 0, nseg = 0;
       bool ok = true;
       while (ok && it.next(p, pre, blockIdx.x, sg)) {
-        if (nseg > 0 && !mbar_wait(bar(kBarQEmpty), (nseg - 1) & 1, ctl)) { ok = false; break; }
-        mbar_expect_tx(bar(kBarQFull), 2u * p.R * 128u);
-        tma_load_3d(sQ, &tmq, bar(kBarQFull), 0, sg.h * p.G, sg.b * p.W);
-        tma_load_3d(sQ + kHalfBytes, &tmq, bar(kBarQFull), 64, sg.h * p.G, sg.b * p.W);
+        const int qs = nseg % qbufs, qu = nseg / qbufs;
+        if (qu > 0 && !mbar_wait(bar(kBarQEmpty + qs), (qu - 1) & 1, ctl)) { ok = false; break; }
+        const uint32_t dq = sQ + qs * 2 * kQHalf;
+        mbar_expect_tx(bar(kBarQFull + qs), 2u * p.R * 128u);
+        tma_load_3d(dq, &tmq, bar(kBarQFull + qs), 0, sg.h * p.G, sg.b * p.W);
+        tma_load_3d(dq + kQHalf, &tmq, bar(kBarQFull + qs), 64, sg.h * p.G, sg.b * p.W);
         const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
         const int nt = tiles_of(sg);
         for (int t = 0; t < nt; ++t, ++g) {
-          const int st = g % kStages, use = g / kStages;
-          if (use > 0 && !mbar_wait(bar(kBarEmpty + st), (use - 1) & 1, ctl)) { ok = false; break; }
-          const uint32_t dk = sStage + st * kStageBytes, dv = dk + kTileBytes;
-          mbar_expect_tx(bar(kBarFull + st), (uint32_t)kStageBytes);
           const int row = row0 + t * kNT;
-          tma_load_2d(dk, &tmk, bar(kBarFull + st), 0, row);
-          tma_load_2d(dk + kHalfBytes, &tmk, bar(kBarFull + st), 64, row);
-          tma_load_2d(dv, &tmv, bar(kBarFull + st), 0, row);
-          tma_load_2d(dv + kHalfBytes, &tmv, bar(kBarFull + st), 64, row);
+          const int ks = g % kKStages, ku = g / kKStages;
+          if (ku > 0 && !mbar_wait(bar(kBarKEmpty + ks), (ku - 1) & 1, ctl)) { ok = false; break; }
+          const uint32_t dk = sK + ks * kTileBytes;
+          mbar_expect_tx(bar(kBarKFull + ks), (uint32_t)kTileBytes);
+          tma_load_2d(dk, &tmk, bar(kBarKFull + ks), 0, row);
+          tma_load_2d(dk + kHalfBytes, &tmk, bar(kBarKFull + ks), 64, row);
         }
         ++nseg;
       }
       // Drain: the copies issued last must have landed before shared memory is released.
-      for (int back = 1; back <= kStages && g - back >= 0; ++back) {
+      for (int back = 1; back <= kKStages && g - back >= 0; ++back) {
         const int gg = g - back;
-        mbar_drain(bar(kBarFull + gg % kStages), (gg / kStages) & 1, 100000000LL);
+        mbar_drain(bar(kBarKFull + gg % kKStages), (gg / kKStages) & 1, 100000000LL);
       }
-      if (nseg > 0) mbar_drain(bar(kBarQFull), (nseg - 1) & 1, 100000000LL);
+      if (nseg > 0) mbar_drain(bar(kBarQFull + (nseg - 1) % qbufs), ((nseg - 1) / qbufs) & 1, 100000000LL);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ TMA producer: V
+    if (lane == 0) {
+      SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
+      Segment sg;
+      int g = 0;
+      bool ok = true;
+      while (ok && it.next(p, pre, blockIdx.x, sg)) {
+        const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
+        const int nt = tiles_of(sg);
+        for (int t = 0; t < nt; ++t, ++g) {
+          const int row = row0 + t * kNT;
+          const int vs = g % vstages, vu = g / vstages;
+          if (vu > 0 && !mbar_wait(bar(kBarVEmpty + vs), (vu - 1) & 1, ctl)) { ok = false; break; }
+          const uint32_t dv = sV + vs * kTileBytes;
+          mbar_expect_tx(bar(kBarVFull + vs), (uint32_t)kTileBytes);
+          tma_load_2d(dv, &tmv, bar(kBarVFull + vs), 0, row);
+          tma_load_2d(dv + kHalfBytes, &tmv, bar(kBarVFull + vs), 64, row);
+        }
+      }
+      for (int back = 1; back <= vstages && g - back >= 0; ++back) {
+        const int gg = g - back;
+        mbar_drain(bar(kBarVFull + gg % vstages), (gg / vstages) & 1, 100000000LL);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -311,52 +429,94 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       Segment sg;
       int g = 0, nseg = 0;
       bool ok = true;
-      const uint64_t sbo = 1024;
+      uint32_t sQseg = sQ;   // Q buffer of the current segment
       auto issue_qk = [&](int gg) {
-        const int st = gg % kStages;
-        const uint32_t d = tmem + (uint32_t)((gg & 1) * kNT);
-        const uint32_t kb = sStage + st * kStageBytes;
+        const uint32_t kb = sK + (gg % kKStages) * kTileBytes;
+        const uint32_t d = tmem + kColS + (uint32_t)((gg % kSBufs) * NQ);
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * kHalfBytes + (kk & 3) * 32);
-          umma(d, sdesc(sQ + off, 16, sbo), sdesc(kb + off, 16, sbo), kIdescQK, kk > 0);
+          const uint32_t ka = kb + (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          const uint32_t qa = sQseg + (kk >> 2) * kQHalf + (kk & 3) * 32;
+          umma(d, sdesc(ka, 16, 1024, 2), sdesc(qa, 16, 1024, 2), kIdescQK, kk > 0);
         }
       };
-      auto issue_pv = [&](int gg) {
-        const int st = gg % kStages;
-        const uint32_t vb = sStage + st * kStageBytes + kTileBytes;
+      auto issue_pv = [&](int gg, bool first) {
+        const uint32_t vb = sV + (gg % vstages) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kNT / 16; ++kk) {
-          const uint64_t bdesc = sdesc(vb + kk * 2048, kHalfBytes, sbo);
-          umma(tmem + kColO, sdesc(sPhi + kk * 32, 16, sbo), bdesc, kIdescPV, kk > 0);
-          umma(tmem + kColO, sdesc(sPlo + kk * 32, 16, sbo), bdesc, kIdescPV, 1);
+          const uint64_t pdesc = sdesc(sP + (gg & 1) * (NQ * 512) + kk * 256, 128, 2048, 0);
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          umma(tmem + kColO, sdesc(vb + kk * 2048, kHalfBytes, 1024, 2), pdesc, kIdescPV, acc);
+          // All-ones A: K-major, no swizzle, every core matrix (8 rows x 16 B) is the same
+          // 128 bytes of ones (leading and stride byte offsets 0).
+          umma(tmem + kColL, sdesc(sOnes, 0, 0, 0), pdesc, kIdescL, acc);
         }
       };
       while (ok && it.next(p, pre, blockIdx.x, sg)) {
         const int nt = tiles_of(sg);
-        if (!mbar_wait(bar(kBarQFull), nseg & 1, ctl)) { ok = false; break; }
+        const int qs = nseg % qbufs;
+        if (!mbar_wait(bar(kBarQFull + qs), (nseg / qbufs) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
+        sQseg = sQ + qs * 2 * kQHalf;
+        // Issue S^T(t) as soon as K(t) has landed and its S buffer is free (P(t-2) consumed),
+        // and O^T += V^T P^T(t) as soon as P(t) and V(t) are ready, whichever comes first.
         const int g0 = g;
-        if (!mbar_wait(bar(kBarFull + g0 % kStages), (g0 / kStages) & 1, ctl)) { ok = false; break; }
-        tc_fence_after();
-        issue_qk(g0);
-        umma_commit(bar(kBarSFull + (g0 & 1)));
-        if (nt == 1) umma_commit(bar(kBarQEmpty));
-        for (int t = 0; t < nt; ++t) {
-          const int gt = g0 + t;
-          if (t + 1 < nt) {
-            const int gn = gt + 1;
-            if (!mbar_wait(bar(kBarFull + gn % kStages), (gn / kStages) & 1, ctl)) { ok = false; break; }
-            tc_fence_after();
-            issue_qk(gn);
-            umma_commit(bar(kBarSFull + (gn & 1)));
-            if (t + 2 == nt) umma_commit(bar(kBarQEmpty));
+        int nqk = 0, npv = 0;
+        long long t_prog = now_ns();
+        uint32_t spins = 0;
+        while (npv < nt) {
+          bool prog = false;
+          const bool want_qk = nqk < nt && nqk <= npv + kSBufs - 1;
+          const bool want_pv = npv < nqk;
+          if (want_qk != want_pv) {
+            // One event pending: a (bounded) blocking wait is cheaper than polling.
+            const bool got = want_qk
+                ? mbar_wait(bar(kBarKFull + (g0 + nqk) % kKStages), ((g0 + nqk) / kKStages) & 1, ctl)
+                : (mbar_wait(bar(kBarPFull + ((g0 + npv) & 1)), ((g0 + npv) >> 1) & 1, ctl) &&
+                   mbar_wait(bar(kBarVFull + (g0 + npv) % vstages), ((g0 + npv) / vstages) & 1, ctl));
+            if (!got) { ok = false; break; }
           }
-          if (!mbar_wait(bar(kBarPFull), gt & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(gt);
-          umma_commit(bar(kBarOFull));
-          umma_commit(bar(kBarEmpty + gt % kStages));
+          if (want_qk) {
+            const int gq = g0 + nqk;
+            if (mbar_test(bar(kBarKFull + gq % kKStages), (gq / kKStages) & 1)) {
+              tc_fence_after();
+              issue_qk(gq);
+              umma_commit(bar(kBarSFull + gq % kSBufs));
+              umma_commit(bar(kBarKEmpty + gq % kKStages));
+              if (nqk == nt - 1) umma_commit(bar(kBarQEmpty + qs));
+              ++nqk;
+              prog = true;
+            }
+          }
+          if (want_pv) {
+            const int gp = g0 + npv;
+            if (mbar_test(bar(kBarPFull + (gp & 1)), (gp >> 1) & 1) &&
+                mbar_test(bar(kBarVFull + gp % vstages), (gp / vstages) & 1)) {
+              tc_fence_after();
+              issue_pv(gp, npv == 0);
+              umma_commit(bar(kBarOFull + (gp & 1)));
+              umma_commit(bar(kBarVEmpty + gp % vstages));
+              ++npv;
+              prog = true;
+            }
+          }
+          if (prog) {
+            spins = 0;
+            t_prog = now_ns();
+            continue;
+          }
+          // Idle poll: back off so this thread does not take issue slots from the softmax
+          // warp that shares its scheduler.
+          __nanosleep(32);
+          if ((++spins & 63u) == 0) {
+            if (*abort_flag) { ok = false; break; }
+            if (now_ns() - t_prog > kWaitLimitNs) {
+              *abort_flag = 1;
+              atomicOr(&p.hdr->err, kErrTimeout);
+              ok = false;
+              break;
+            }
+          }
         }
         g = g0 + nt;
         ++nseg;
@@ -367,200 +527,285 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
-    const int q4 = warp & 3;
-    const int t0 = lane & 3, t1 = lane >> 2;
-    const int ra = 16 * q4 + t1, rb = ra + 8;
-    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    const int stid = tid - 64;  // 0..127
+    // Per tile each thread holds its key's NQ scores. The per-row references m (log2 units,
+    // shared by all threads) live in shared memory, double-buffered; row sums accumulate in
+    // TMEM next to O.
+    const int sub = warp & 3;                   // TMEM sub-partition of this warp
+    const int w4 = warp - 2;                    // 0..3 within the softmax group
+    const int row = 32 * sub + lane;            // key of the S^T tile / channel of O^T
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * sub) << 16);
+    const int stid = tid - 64;                  // 0..127
+    float* rowst = reinterpret_cast<float*>(base + L.mref);   // [2][NQ]
+    const float c2 = p.scale_log2;
     SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
     Segment sg;
     int g = 0;
     bool ok = true;
     while (ok && it.next(p, pre, blockIdx.x, sg)) {
       const int nt = tiles_of(sg);
-      const int lim_a = (ra < p.R) ? min(row_limit(p, sg.n, ra), sg.j1) : 0;
-      const int lim_b = (rb < p.R) ? min(row_limit(p, sg.n, rb), sg.j1) : 0;
-      float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-      float alpha_a = 0.f, alpha_b = 0.f;
-      float o[64];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) o[i] = 0.f;
-
-      auto fold_o = [&](int gg, float aa, float ab) -> bool {
-        if (!mbar_wait(bar(kBarOFull), gg & 1, ctl)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[16];
-          tmem_ld_x4(tmem + lane_base + kColO + 32 * c, v);
-          tc_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int i = 16 * c + 4 * k;
-            o[i + 0] = fmaf(o[i + 0], aa, v[4 * k + 0]);
-            o[i + 1] = fmaf(o[i + 1], aa, v[4 * k + 1]);
-            o[i + 2] = fmaf(o[i + 2], ab, v[4 * k + 2]);
-            o[i + 3] = fmaf(o[i + 3], ab, v[4 * k + 3]);
-          }
-        }
-        return true;
-      };
+      for (int q = stid; q < NQ; q += 128) {
+        if (CAUSAL) lim_s[2 * NQ + q] = (q < p.R) ? min(row_limit(p, sg.n, q), sg.j1) : 0;
+        rowst[q] = -INFINITY;            // no reference yet
+      }
+      softmax_bar();
+      const int* lim_q = lim_s + 2 * NQ;
+      int cur = 0;
 
       for (int t = 0; t < nt; ++t) {
         const int gt = g + t;
         const int jt = sg.j0 + t * kNT;
-        if (!mbar_wait(bar(kBarSFull + (gt & 1)), (gt >> 1) & 1, ctl)) { ok = false; break; }
+        const int key = jt + row;
+        const bool key_ok = key < sg.j1;
+        const uint32_t s_addr = lane_addr + kColS + (gt % kSBufs) * NQ;
+        if (!mbar_wait(bar(kBarSFull + gt % kSBufs), (gt / kSBufs) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
-        float s[32];
-        tmem_ld_x8(tmem + lane_base + (uint32_t)((gt & 1) * kNT), s);
+        float x[NQ];
+#pragma unroll
+        for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
         tc_wait_ld();
-
-        // Mask and row maxima (log2 domain). Column of s[4k+e]: 8k + 2*t0 + (e & 1).
-        float mx_a = -INFINITY, mx_b = -INFINITY;
+        // y = score * scale_log2 - reference: the vote asks whether some y exceeds the lazy
+        // threshold, and p = 2^y against the current references (a row without a reference
+        // yet has m = -inf, so y = +inf votes for a rescale). Padding rows (q >= R) need no
+        // mask: their Q rows are zero, so their scores are exactly 0.
+        const float4* mr4 = reinterpret_cast<const float4*>(rowst + cur * NQ);
+        bool exceeds = false;
+        if (CAUSAL || key_ok) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+          for (int c4 = 0; c4 < NQ / 4; ++c4) {
+            const float4 m4 = mr4[c4];
+            const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = jt + 8 * k + 2 * t0 + e;
-            float xa = (j < lim_a) ? s[4 * k + e] * p.scale_log2 : -INFINITY;
-            float xb = (j < lim_b) ? s[4 * k + 2 + e] * p.scale_log2 : -INFINITY;
-            s[4 * k + e] = xa;
-            s[4 * k + 2 + e] = xb;
-            mx_a = fmaxf(mx_a, xa);
-            mx_b = fmaxf(mx_b, xb);
+            for (int e = 0; e < 4; ++e) {
+              const int q = 4 * c4 + e;
+              const float y = fmaf(x[q], c2, -mq[e]);
+              const bool v = CAUSAL ? (key < lim_q[q]) : true;
+              exceeds |= v && (y > kLazyThreshold);
+              x[q] = v ? fast_exp2(y) : 0.f;
+            }
           }
+        } else {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) x[q] = 0.f;
         }
-        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-        const float na = (mn_a == -INFINITY) ? 1.f : fast_exp2(m_a - mn_a);
-        const float nb = (mn_b == -INFINITY) ? 1.f : fast_exp2(m_b - mn_b);
-        const float ref_a = (mn_a == -INFINITY) ? 0.f : mn_a;
-        const float ref_b = (mn_b == -INFINITY) ? 0.f : mn_b;
-        m_a = mn_a;
-        m_b = mn_b;
-        float sum_a = 0.f, sum_b = 0.f;
+        // CTA-wide vote: raise the references only if some score is far above them.
+        const bool rescale = softmax_bar_or(exceeds);
+        if (rescale) {
+          // Exact tile maxima per row (log2 units): warp reduction, then across the warps.
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+          for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
+          tc_wait_ld();
+          float* wm = wmax + (gt & 1) * 4 * NQ;
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float pa = fast_exp2(s[4 * k + e] - ref_a);
-            const float pb = fast_exp2(s[4 * k + 2 + e] - ref_b);
-            s[4 * k + e] = pa;
-            s[4 * k + 2 + e] = pb;
-            sum_a += pa;
-            sum_b += pb;
+          for (int q = 0; q < NQ; ++q) {
+            const bool v = CAUSAL ? (key < lim_q[q]) : key_ok;
+            x[q] = v ? x[q] * c2 : -INFINITY;
+            const float m = warp_max_f32(x[q]);
+            if ((q & 31) == lane) wm[w4 * NQ + q] = m;
           }
-        }
-        l_a = l_a * na + sum_a;
-        l_b = l_b * nb + sum_b;
-
-        // Fold the previous tile's PV (its P buffer is then free), remember this tile's alpha.
-        if (t > 0 && !fold_o(gt - 1, alpha_a, alpha_b)) { ok = false; break; }
-        alpha_a = na;
-        alpha_b = nb;
-
-        // P = P_hi + P_lo as bf16 into the swizzled K-major operand tiles.
+          softmax_bar();
+          // The previous PV product (and so every earlier one) must be complete before O and l
+          // are rescaled in place.
+          if (gt > 0) {
+            if (!mbar_wait(bar(kBarOFull + ((gt - 1) & 1)), ((gt - 1) >> 1) & 1, ctl)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const float* mo_s = rowst + cur * NQ;
+          float* mw = rowst + (cur ^ 1) * NQ;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          __nv_bfloat162 ha = __floats2bfloat162_rn(s[4 * k + 0], s[4 * k + 1]);
-          __nv_bfloat162 hb = __floats2bfloat162_rn(s[4 * k + 2], s[4 * k + 3]);
-          float2 fa = __bfloat1622float2(ha), fb = __bfloat1622float2(hb);
-          __nv_bfloat162 la2 = __floats2bfloat162_rn(s[4 * k + 0] - fa.x, s[4 * k + 1] - fa.y);
-          __nv_bfloat162 lb2 = __floats2bfloat162_rn(s[4 * k + 2] - fb.x, s[4 * k + 3] - fb.y);
-          const uint32_t offa = (uint32_t)(ra * 128 + ((k ^ (ra & 7)) << 4) + 4 * t0);
-          const uint32_t offb = (uint32_t)(rb * 128 + ((k ^ (rb & 7)) << 4) + 4 * t0);
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sPhi + offa), "r"(pack_bf16x2(ha)));
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sPhi + offb), "r"(pack_bf16x2(hb)));
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sPlo + offa), "r"(pack_bf16x2(la2)));
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sPlo + offb), "r"(pack_bf16x2(lb2)));
+          for (int c = 0; c < NQ / 16; ++c) {
+            float al[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int q = 16 * c + e;
+              const float tm = fmaxf(fmaxf(wm[q], wm[NQ + q]), fmaxf(wm[2 * NQ + q], wm[3 * NQ + q]));
+              const float mo = mo_s[q];
+              const float mn = fmaxf(mo, tm);
+              const float safe = (mn == -INFINITY) ? 0.f : mn;
+              al[e] = (mn == -INFINITY) ? 1.f : fast_exp2(mo - mn);
+              if (q == stid) mw[q] = mn;
+              x[q] = fast_exp2(x[q] - safe);
+            }
+            if (t > 0) {
+              // O hi, O lo, l hi, l lo columns of rows 16c..16c+15.
+#pragma unroll
+              for (int blk = 0; blk < 4; ++blk) {
+                float o[16];
+                const uint32_t col = kColO + blk * NQ + 16 * c;
+                tmem_ld16(lane_addr + col, o);
+                tc_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) o[e] *= al[e];
+                tmem_st16(lane_addr + col, o);
+              }
+            }
+          }
+          if (t > 0) tc_wait_st();
+          // The new references must be visible to every thread before the next tile reads them.
+          softmax_bar();
+          cur ^= 1;
+        } else if (gt > 1) {
+          // The product that read this P^T buffer two tiles ago must be done.
+          if (!mbar_wait(bar(kBarOFull + (gt & 1)), ((gt - 2) >> 1) & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+        }
+
+        // P^T as hi/lo row groups (one 16-byte store per 8 rows).
+        const uint32_t prow = sP + (gt & 1) * (NQ * 512) + (uint32_t)((row >> 3) * 128 + (row & 7) * 16);
+#pragma unroll
+        for (int m = 0; m < NQ / 8; ++m) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a = x[8 * m + 2 * e], b = x[8 * m + 2 * e + 1];
+            hi[e] = pack_bf16x2(a, b);
+            const float ha = __uint_as_float(hi[e] << 16), hb = __uint_as_float(hi[e] & 0xFFFF0000u);
+            lo[e] = pack_bf16x2(a - ha, b - hb);
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + m * 2048), "r"(hi[0]),
+                       "r"(hi[1]), "r"(hi[2]), "r"(hi[3]));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + (NQ / 8 + m) * 2048),
+                       "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]));
         }
         // Rows of the V tile past the segment end hold other data: zero them so 0 * x
         // cannot turn into NaN in the tensor-core product.
         const int valid = min(kNT, sg.j1 - jt);
         if (valid < kNT) {
-          const uint32_t vb = sStage + (gt % kStages) * kStageBytes + kTileBytes;
+          // The tile's V copy must have landed before its tail is overwritten.
+          if (!mbar_wait(bar(kBarVFull + gt % vstages), (gt / vstages) & 1, ctl)) { ok = false; break; }
+          const uint32_t vbase = sV + (gt % vstages) * kTileBytes;
           for (int idx = stid; idx < (kNT - valid) * 16; idx += 128) {
-            const int row = valid + (idx >> 4), ch = idx & 15;
-            const uint32_t a = vb + (ch >> 3) * kHalfBytes + row * 128 + (ch & 7) * 16;
+            const int r = valid + (idx >> 4), ch = idx & 15;
+            const uint32_t a = vbase + (ch >> 3) * kHalfBytes + r * 128 + (ch & 7) * 16;
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(0u), "r"(0u),
                          "r"(0u), "r"(0u));
           }
         }
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(kBarPFull));
+        mbar_arrive(bar(kBarPFull + (gt & 1)));
       }
       if (!ok) break;
-      if (!fold_o(g + nt - 1, alpha_a, alpha_b)) { ok = false; break; }
+      const int glast = g + nt - 1;
       g += nt;
+      if (!mbar_wait(bar(kBarOFull + (glast & 1)), (glast >> 1) & 1, ctl)) { ok = false; break; }
+      tc_fence_after();
 
-      // Row sums across the quad, then the output or the partial.
-      l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-      l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+      // Epilogue: O^T row `row` (one channel) and the row sums (identical in every lane) are
+      // staged in the idle P^T buffer as [R][128] (bf16 output rows, or fp32 partial rows)
+      // and written by one asynchronous TMA store, so the warps do not stall on global
+      // stores while the memory system is saturated by the K/V stream.
+      float* slot = sg.whole ? nullptr : slot_ptr(p, sg.slot);
+      const uint32_t stg = sP;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r = half ? rb : ra;
-        if (r >= p.R) continue;
-        const float l = half ? l_b : l_a;
-        const float m = half ? m_b : m_a;
-        if (sg.whole) {
-          const float inv = 1.f / l;
-          __nv_bfloat16* dst = p.out + out_row_offset(p, sg.b, sg.h, r);
+      for (int c = 0; c < NQ / 16; ++c) {
+        float ohi[16], olo[16], lhi[16], llo[16];
+        tmem_ld16(lane_addr + kColO + 16 * c, ohi);
+        tmem_ld16(lane_addr + kColO + NQ + 16 * c, olo);
+        tmem_ld16(lane_addr + kColL + 16 * c, lhi);
+        tmem_ld16(lane_addr + kColL + NQ + 16 * c, llo);
+        tc_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int d = 8 * k + 2 * t0;
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(o[4 * k + 2 * half] * inv,
-                                                      o[4 * k + 2 * half + 1] * inv);
-            *reinterpret_cast<__nv_bfloat162*>(dst + d) = v2;
-          }
-        } else {
-          float* slot = slot_ptr(p, sg.slot);
-          if (t0 == 0) {
-            slot[r] = m;
-            slot[p.rows_pad + r] = l;
-          }
-          float* acc = slot + 2 * p.rows_pad + (size_t)r * kHeadDim;
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int d = 8 * k + 2 * t0;
-            *reinterpret_cast<float2*>(acc + d) = make_float2(o[4 * k + 2 * half], o[4 * k + 2 * half + 1]);
+        for (int e = 0; e < 16; ++e) {
+          const int q = 16 * c + e;
+          if (q >= p.R) continue;
+          const float o = ohi[e] + olo[e], l = lhi[e] + llo[e];
+          if (sg.whole) {
+            const __nv_bfloat16 v = __float2bfloat16_rn(o / l);
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 2u),
+                         "h"(*reinterpret_cast<const unsigned short*>(&v)));
+          } else {
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 4u), "f"(o));
+            if (q == stid) {
+              slot[q] = rowst[cur * NQ + q];
+              slot[p.rows_pad + q] = l;
+            }
           }
         }
       }
+      fence_async_smem();
+      softmax_bar();
+      if (stid == 0) {
+        if (sg.whole) {
+          asm volatile(
+              "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                  reinterpret_cast<uint64_t>(&tmo)),
+              "r"(stg), "r"(0), "r"(sg.h * p.G), "r"(sg.b * p.W)
+              : "memory");
+        } else {
+          asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                           slot + 2 * p.rows_pad),
+                       "r"(stg), "r"(p.R * kHeadDim * 4)
+                       : "memory");
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        // The staging buffer is reused as P^T by the next segment: wait until it was read.
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      }
+      // O, l and the shared per-segment buffers are reused by the next segment.
+      tc_fence_before();
+      softmax_bar();
     }
   }
 
+  // Epilogue stores issued by this thread must be complete before the CTA retires.
+  if (tid == 64) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
   }
 }
 
-int tc_ctas_per_sm() { return 2; }
+int tc_ctas_per_sm() { return 1; }
 int tc_min_chunk() { return kNT; }
 
-size_t tc_smem_bytes(int B) {
-  const size_t pre_ints = (size_t)round_up(B + 1, 4) + 32;
-  return 1024 + kOffPre + pre_ints * 4;
+static int tc_nq(int R) { return round_up(R, 16); }
+
+// V ring depth and Q buffers that fit: the V ring depth matters most (a V tile is held until
+// its PV product completes), a second Q buffer only hides segment changes.
+static int tc_ring(int nq, int B) {
+  const int limit = 227 * 1024 - 1024;
+  const int options[5][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}, {1, 1}};
+  for (auto& o : options)
+    if (tc_layout(nq, o[0], o[1], B).end <= limit) return o[0] | (o[1] << 8);
+  return 0;
+}
+
+size_t tc_smem_bytes(int R, int B) {
+  const int nq = tc_nq(R);
+  const int ring = tc_ring(nq, B);
+  return ring ? (size_t)1024 + tc_layout(nq, ring & 0xff, ring >> 8, B).end : 0;
+}
+
+template <int NQ, bool CAUSAL>
+static cudaError_t launch_nq(const Problem& p, const CUtensorMap& k, const CUtensorMap& v,
+                             const CUtensorMap& q, const CUtensorMap& o, cudaStream_t stream) {
+  const int ring = tc_ring(NQ, p.B);
+  if (ring == 0) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)1024 + tc_layout(NQ, ring & 0xff, ring >> 8, p.B).end;
+  cudaError_t e = cudaFuncSetAttribute(pbd_attn_tc_kernel<NQ, CAUSAL>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  pbd_attn_tc_kernel<NQ, CAUSAL><<<p.num_ctas, kThreadsTc, smem, stream>>>(k, v, q, o, p, ring);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tmap_v,
-                           const void* tmap_q, cudaStream_t stream) {
-  const size_t smem = tc_smem_bytes(p.B);
-  cudaError_t e = cudaFuncSetAttribute(pbd_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  pbd_attn_tc_kernel<<<p.num_ctas, kThreadsTc, smem, stream>>>(
-      *static_cast<const CUtensorMap*>(tmap_k), *static_cast<const CUtensorMap*>(tmap_v),
-      *static_cast<const CUtensorMap*>(tmap_q), p);
-  return cudaGetLastError();
+                           const void* tmap_q, const void* tmap_o, cudaStream_t stream) {
+  const CUtensorMap& k = *static_cast<const CUtensorMap*>(tmap_k);
+  const CUtensorMap& v = *static_cast<const CUtensorMap*>(tmap_v);
+  const CUtensorMap& q = *static_cast<const CUtensorMap*>(tmap_q);
+  const CUtensorMap& o = *static_cast<const CUtensorMap*>(tmap_o);
+  const bool causal = p.mask_mode != 0;
+  switch (tc_nq(p.R)) {
+    case 16: return causal ? launch_nq<16, true>(p, k, v, q, o, stream) : launch_nq<16, false>(p, k, v, q, o, stream);
+    case 32: return causal ? launch_nq<32, true>(p, k, v, q, o, stream) : launch_nq<32, false>(p, k, v, q, o, stream);
+    case 48: return causal ? launch_nq<48, true>(p, k, v, q, o, stream) : launch_nq<48, false>(p, k, v, q, o, stream);
+    case 64: return causal ? launch_nq<64, true>(p, k, v, q, o, stream) : launch_nq<64, false>(p, k, v, q, o, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace la

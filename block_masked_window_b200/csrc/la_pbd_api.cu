@@ -6,7 +6,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/la_pbd.h"
+#include "la_pbd.h"
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 #include "tma_util.h"
@@ -186,7 +186,7 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
     if (la::make_tma_maps(p, &maps) != cudaSuccess) return LA_ERR_CUDA;
     p.c_min = la::tc_min_chunk();
     p.num_ctas = grid_for(p, sms * la::tc_ctas_per_sm());
-    e = la::launch_attn_tc(p, &maps.k, &maps.v, &maps.q, s);
+    e = la::launch_attn_tc(p, &maps.k, &maps.v, &maps.q, &maps.o, s);
   } else {
     int per_sm = 0;
     e = la::simt_max_ctas_per_sm(p.R, p.B, &per_sm);

@@ -12,7 +12,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/la_pbd.h"
+#include "la_pbd.h"
 
 namespace {
 

@@ -17,12 +17,13 @@
 
 namespace la {
 
-constexpr int kTileKeys = 64;  // keys per tile of the tcgen05 kernel
+constexpr int kTileKeys = 128;  // keys per tile of the tcgen05 kernel
 
 struct TmaMaps {
   alignas(64) CUtensorMap k;
   alignas(64) CUtensorMap v;
   alignas(64) CUtensorMap q;
+  alignas(64) CUtensorMap o;   // output rows, store map (no swizzle, whole 256-byte rows)
 };
 
 int tc_ctas_per_sm();
@@ -68,6 +69,12 @@ inline cudaError_t make_tma_maps(const Problem& p, TmaMaps* m) {
     CUresult r = enc(&m->q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)p.q, dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // Same geometry over `out`, whole 128-channel rows, for the epilogue's TMA stores.
+    cuuint32_t obox[3] = {(cuuint32_t)kHeadDim, (cuuint32_t)p.G, (cuuint32_t)p.W};
+    r = enc(&m->o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)p.out, dims, strides, obox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   }
   return cudaSuccess;
