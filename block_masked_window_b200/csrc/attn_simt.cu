@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(kThreads) pbd_attn_simt_kernel(Problem p) {
   constexpr int ROWS = 16 * RPT;
   constexpr int PROWS = 2 * RPT;  // rows per thread in the PV phase
 
+  pdl_trigger();
+  pdl_wait();
   plan_prefix(p, s.pre, s.warp_tot);
   __syncthreads();
   const long long T = (long long)p.Hkv * s.pre[p.B];
@@ -304,8 +306,7 @@ cudaError_t launch_rpt(const Problem& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(pbd_attn_simt_kernel<RPT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  pbd_attn_simt_kernel<RPT><<<p.num_ctas, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(pbd_attn_simt_kernel<RPT>, dim3(p.num_ctas), dim3(kThreads), smem, stream, p);
 }
 
 template <int RPT>

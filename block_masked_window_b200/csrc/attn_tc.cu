@@ -78,7 +78,7 @@ constexpr int kNumBars = kBarDrain + 1;
 
 // Shared-memory plan for a given NQ and V ring depth.
 struct TcLayout {
-  int k, v, q, p, ones, bar, misc, vote, wmax, lim, mref, pre, end;
+  int k, v, q, p, ones, bar, misc, vote, wmax, lim, mref, alpha, pre, end;
 };
 __host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, int B) {
   // Operand buffers are 1024-byte multiples from a 1024-aligned base; every small region is
@@ -96,7 +96,8 @@ __host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, in
   L.wmax = L.vote + 32;                     // [2][4][nq] floats
   L.lim = a16(L.wmax + 2 * 4 * nq * 4);     // [3][nq] ints: (unused), output offsets, key limits
   L.mref = a16(L.lim + 3 * nq * 4);         // [2][nq]: per-row references
-  L.pre = a16(L.mref + 2 * nq * 4);         // [B+1] + 32 ints
+  L.alpha = a16(L.mref + 2 * nq * 4);       // [nq]: rescale factors of the last reference update
+  L.pre = a16(L.alpha + nq * 4);            // [B+1] + 32 ints
   L.end = L.pre + (round_up(B + 1, 4) + 32) * 4;
   return L;
 }
@@ -316,6 +317,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Ctl ctl{abort_flag, p.hdr};
+  pdl_trigger();
+  if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmq)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmo)) : "memory");
+  }
 
   // Q rows R..NQ-1 must read as zero: clear both Q buffers once (TMA rewrites rows < R).
   for (int i = tid; i < 4 * kQHalf / 16; i += kThreadsTc)
@@ -350,6 +358,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  // Everything above is on-chip; from here on global memory written by the previous kernel
+  // of the stream is read.
+  pdl_wait();
   plan_prefix(p, pre, warp_tot);
   fence_async_smem();
   tc_fence_before();
@@ -536,6 +547,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * sub) << 16);
     const int stid = tid - 64;                  // 0..127
     float* rowst = reinterpret_cast<float*>(base + L.mref);   // [2][NQ]
+    float* alpha_s = reinterpret_cast<float*>(base + L.alpha); // [NQ]
     const float c2 = p.scale_log2;
     SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
     Segment sg;
@@ -563,37 +575,43 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
         for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
         tc_wait_ld();
-        // y = score * scale_log2 - reference: the vote asks whether some y exceeds the lazy
-        // threshold, and p = 2^y against the current references (a row without a reference
-        // yet has m = -inf, so y = +inf votes for a rescale). Padding rows (q >= R) need no
-        // mask: their Q rows are zero, so their scores are exactly 0.
-        const float4* mr4 = reinterpret_cast<const float4*>(rowst + cur * NQ);
-        bool exceeds = false;
-        if (CAUSAL || key_ok) {
+        // A segment's first tile has no references yet: it always takes the exact-maximum
+        // path below, with the raw scores still in x.
+        bool rescale = true;
+        if (t > 0) {
+          // y = score * scale_log2 - reference: the vote asks whether some y exceeds the lazy
+          // threshold, and p = 2^y against the current references. Padding rows (q >= R)
+          // need no mask: their Q rows are zero, so their scores are exactly 0.
+          const float4* mr4 = reinterpret_cast<const float4*>(rowst + cur * NQ);
+          bool exceeds = false;
+          if (CAUSAL || key_ok) {
 #pragma unroll
-          for (int c4 = 0; c4 < NQ / 4; ++c4) {
-            const float4 m4 = mr4[c4];
-            const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
+            for (int c4 = 0; c4 < NQ / 4; ++c4) {
+              const float4 m4 = mr4[c4];
+              const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int q = 4 * c4 + e;
-              const float y = fmaf(x[q], c2, -mq[e]);
-              const bool v = CAUSAL ? (key < lim_q[q]) : true;
-              exceeds |= v && (y > kLazyThreshold);
-              x[q] = v ? fast_exp2(y) : 0.f;
+              for (int e = 0; e < 4; ++e) {
+                const int q = 4 * c4 + e;
+                const float y = fmaf(x[q], c2, -mq[e]);
+                const bool v = CAUSAL ? (key < lim_q[q]) : true;
+                exceeds |= v && (y > kLazyThreshold);
+                x[q] = v ? fast_exp2(y) : 0.f;
+              }
             }
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) x[q] = 0.f;
+            for (int q = 0; q < NQ; ++q) x[q] = 0.f;
+          }
+          // CTA-wide vote: raise the references only if some score is far above them.
+          rescale = softmax_bar_or(exceeds);
+          if (rescale) {
+#pragma unroll
+            for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
+            tc_wait_ld();
+          }
         }
-        // CTA-wide vote: raise the references only if some score is far above them.
-        const bool rescale = softmax_bar_or(exceeds);
         if (rescale) {
           // Exact tile maxima per row (log2 units): warp reduction, then across the warps.
-#pragma unroll
-          for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
-          tc_wait_ld();
           float* wm = wmax + (gt & 1) * 4 * NQ;
 #pragma unroll
           for (int q = 0; q < NQ; ++q) {
@@ -603,30 +621,46 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             if ((q & 31) == lane) wm[w4 * NQ + q] = m;
           }
           softmax_bar();
+          // Thread q publishes the new reference of row q and the factor that rescales what
+          // was accumulated against the old one.
+          float* mw = rowst + (cur ^ 1) * NQ;
+          if (stid < NQ) {
+            const int q = stid;
+            const float tm = fmaxf(fmaxf(wm[q], wm[NQ + q]), fmaxf(wm[2 * NQ + q], wm[3 * NQ + q]));
+            const float mo = rowst[cur * NQ + q];
+            const float mn = fmaxf(mo, tm);
+            mw[q] = mn;
+            alpha_s[q] = (mn == -INFINITY) ? 1.f : fast_exp2(mo - mn);
+          }
           // The previous PV product (and so every earlier one) must be complete before O and l
           // are rescaled in place.
           if (gt > 0) {
             if (!mbar_wait(bar(kBarOFull + ((gt - 1) & 1)), ((gt - 1) >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
           }
-          const float* mo_s = rowst + cur * NQ;
-          float* mw = rowst + (cur ^ 1) * NQ;
+          softmax_bar();
+          const float4* mn4 = reinterpret_cast<const float4*>(mw);
 #pragma unroll
-          for (int c = 0; c < NQ / 16; ++c) {
-            float al[16];
+          for (int c4 = 0; c4 < NQ / 4; ++c4) {
+            const float4 m4 = mn4[c4];
+            const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int q = 16 * c + e;
-              const float tm = fmaxf(fmaxf(wm[q], wm[NQ + q]), fmaxf(wm[2 * NQ + q], wm[3 * NQ + q]));
-              const float mo = mo_s[q];
-              const float mn = fmaxf(mo, tm);
-              const float safe = (mn == -INFINITY) ? 0.f : mn;
-              al[e] = (mn == -INFINITY) ? 1.f : fast_exp2(mo - mn);
-              if (q == stid) mw[q] = mn;
-              x[q] = fast_exp2(x[q] - safe);
+            for (int e = 0; e < 4; ++e) {
+              const float safe = (mq[e] == -INFINITY) ? 0.f : mq[e];
+              x[4 * c4 + e] = fast_exp2(x[4 * c4 + e] - safe);
             }
-            if (t > 0) {
-              // O hi, O lo, l hi, l lo columns of rows 16c..16c+15.
+          }
+          if (t > 0) {
+            // O hi, O lo, l hi, l lo columns, 16 rows at a time.
+            const float4* al4 = reinterpret_cast<const float4*>(alpha_s);
+#pragma unroll
+            for (int c = 0; c < NQ / 16; ++c) {
+              float al[16];
+#pragma unroll
+              for (int e4 = 0; e4 < 4; ++e4) {
+                const float4 a4 = al4[4 * c + e4];
+                al[4 * e4] = a4.x; al[4 * e4 + 1] = a4.y; al[4 * e4 + 2] = a4.z; al[4 * e4 + 3] = a4.w;
+              }
 #pragma unroll
               for (int blk = 0; blk < 4; ++blk) {
                 float o[16];
@@ -638,10 +672,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_st16(lane_addr + col, o);
               }
             }
+            tc_wait_st();
           }
-          if (t > 0) tc_wait_st();
-          // The new references must be visible to every thread before the next tile reads them.
-          softmax_bar();
+          // Nobody reads the old references after the barrier above, and the next writer of
+          // this buffer waits at the next tile's vote barrier.
           cur ^= 1;
         } else if (gt > 1) {
           // The product that read this P^T buffer two tiles ago must be done.
@@ -696,6 +730,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       // stores while the memory system is saturated by the K/V stream.
       float* slot = sg.whole ? nullptr : slot_ptr(p, sg.slot);
       const uint32_t stg = sP;
+      float l_own = 0.f;   // row sum of row q = stid (every lane holds every row's sum)
 #pragma unroll
       for (int c = 0; c < NQ / 16; ++c) {
         float ohi[16], olo[16], lhi[16], llo[16];
@@ -704,23 +739,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         tmem_ld16(lane_addr + kColL + 16 * c, lhi);
         tmem_ld16(lane_addr + kColL + NQ + 16 * c, llo);
         tc_wait_ld();
+        // All 16 values first, then the stores, so the divisions overlap.
+        float res[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int q = 16 * c + e;
-          if (q >= p.R) continue;
           const float o = ohi[e] + olo[e], l = lhi[e] + llo[e];
-          if (sg.whole) {
-            const __nv_bfloat16 v = __float2bfloat16_rn(o / l);
+          if (16 * c + e == stid) l_own = l;
+          res[e] = sg.whole ? o / l : o;
+        }
+        if (sg.whole) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int q = 16 * c + e;
+            if (q >= p.R) break;
+            const __nv_bfloat16 v = __float2bfloat16_rn(res[e]);
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 2u),
                          "h"(*reinterpret_cast<const unsigned short*>(&v)));
-          } else {
-            asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 4u), "f"(o));
-            if (q == stid) {
-              slot[q] = rowst[cur * NQ + q];
-              slot[p.rows_pad + q] = l;
-            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int q = 16 * c + e;
+            if (q >= p.R) break;
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 4u), "f"(res[e]));
           }
         }
+      }
+      if (!sg.whole && stid < p.R) {
+        slot[stid] = rowst[cur * NQ + stid];
+        slot[p.rows_pad + stid] = l_own;
       }
       fence_async_smem();
       softmax_bar();
@@ -788,8 +835,8 @@ static cudaError_t launch_nq(const Problem& p, const CUtensorMap& k, const CUten
   cudaError_t e = cudaFuncSetAttribute(pbd_attn_tc_kernel<NQ, CAUSAL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  pbd_attn_tc_kernel<NQ, CAUSAL><<<p.num_ctas, kThreadsTc, smem, stream>>>(k, v, q, o, p, ring);
-  return cudaGetLastError();
+  return launch_pdl(pbd_attn_tc_kernel<NQ, CAUSAL>, dim3(p.num_ctas), dim3(kThreadsTc), smem,
+                    stream, k, v, q, o, p, ring);
 }
 
 cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tmap_v,

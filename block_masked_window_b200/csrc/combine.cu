@@ -20,6 +20,8 @@ constexpr int kCombineMaxSlots = 1024;   // >= partials of one sequence (<= grid
 
 __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem p) {
   __shared__ float s_w[kCombineRows][kCombineMaxSlots];
+  pdl_trigger();
+  pdl_wait();
   const int s = blockIdx.y;            // sequence = b * Hkv + h
   const int b = s / p.Hkv, h = s - b * p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -92,8 +94,7 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream) {
   if (p.num_ctas > kCombineMaxSlots) return cudaErrorInvalidValue;
   dim3 grid((p.R + kCombineRows - 1) / kCombineRows, p.B * p.Hkv);
-  pbd_combine_kernel<<<grid, 32 * kCombineRows, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(pbd_combine_kernel, grid, dim3(32 * kCombineRows), 0, stream, p);
 }
 
 }  // namespace la

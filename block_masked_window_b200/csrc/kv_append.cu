@@ -13,6 +13,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
     const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_cache,
     uint4* __restrict__ v_cache, const int32_t* __restrict__ seq_lens, int B, int W, int Hkv,
     int S) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const long long rows = (long long)B * W * Hkv;
@@ -39,10 +41,10 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache
   const long long rows = (long long)B * W * Hkv;
   const int warps_per_block = 8;
   const unsigned grid = (unsigned)((rows + warps_per_block - 1) / warps_per_block);
-  kv_append_kernel<<<grid, 32 * warps_per_block, 0, stream>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), seq_lens, B, W, Hkv, S);
-  return cudaGetLastError();
+  return launch_pdl(kv_append_kernel, dim3(grid), dim3(32 * warps_per_block), 0, stream,
+                    static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                    static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), seq_lens, B, W,
+                    Hkv, S);
 }
 
 }  // namespace la

@@ -178,6 +178,15 @@ __device__ inline int row_limit(const Problem& p, int n, int r) {
   return n - p.W + i + 1;
 }
 
+// Programmatic dependent launch. Every kernel of the library is launched so that it may start
+// while the previous kernel of the stream is still running; it signals right away that its own
+// successor may start too, and waits for its predecessor (completion and memory visibility)
+// before the first access to global memory. Every CTA executes the wait before it can exit,
+// so a kernel completes only after its predecessor did: the ordering is transitive along the
+// stream. Launched without the attribute, both instructions are no-ops.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ inline float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
