@@ -16,7 +16,8 @@ __all__ = [
     "LA_MASK_PBD", "LA_MASK_CAUSAL_WINDOW", "LA_ALGO_AUTO", "LA_ALGO_TCGEN05", "LA_ALGO_SIMT",
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
-    "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "Workspace", "EXPORTED_SYMBOLS",
+    "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "Workspace",
+    "EXPORTED_SYMBOLS",
 ]
 
 LA_MASK_PBD = 0
@@ -26,13 +27,14 @@ LA_ALGO_TCGEN05 = 1
 LA_ALGO_SIMT = 2
 
 LA_OK = 0
+LA_ERR_INVALID_ARG_CODE = 1
 STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
                 3: "LA_ERR_WORKSPACE", 4: "LA_ERR_CUDA", 5: "LA_ERR_SEQ_OVERFLOW",
                 6: "LA_ERR_TIMEOUT"}
 
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
-                    "la_pbd_check", "la_pbd_attn_static"]
+                    "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: Optional[ctypes.CDLL] = None
@@ -94,6 +96,8 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_check.argtypes = [vp, vp]
     lib.la_pbd_attn_static.restype = i32
     lib.la_pbd_attn_static.argtypes = [cfgp, vp, vp, vp, vp, i32, vp, vp]
+    lib.la_pbd_plan.restype = i32
+    lib.la_pbd_plan.argtypes = [cfgp, i32, vp, i32, i32, vp, i32]
     _LIB = lib
     return lib
 
@@ -235,3 +239,20 @@ def la_pbd_attn_static(cfg: Config, q, k_cache, v_cache, seq_lens, window_len: i
     _check(load().la_pbd_attn_static(ctypes.byref(cfg), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                      _ptr(seq_lens), W, _ptr(out), _stream(stream)),
            "la_pbd_attn_static")
+
+
+def la_pbd_plan(cfg: Config, window_len: int, seq_lens, num_ctas: int, unit_keys: int):
+    """Host-side split-KV work plan (no GPU work): a list of (cta, b, h, j0, j1, slot)
+    tuples in CTA order; slot is -1 for a segment that is a whole sequence."""
+    lens = (ctypes.c_int32 * cfg.batch)(*[int(x) for x in seq_lens])
+    lib = load()
+    n = lib.la_pbd_plan(ctypes.byref(cfg), int(window_len), ctypes.cast(lens, ctypes.c_void_p),
+                        int(num_ctas), int(unit_keys), None, 0)
+    if n < 0:
+        raise LaError(-n, "la_pbd_plan")
+    buf = (ctypes.c_int32 * (6 * max(n, 1)))()
+    m = lib.la_pbd_plan(ctypes.byref(cfg), int(window_len), ctypes.cast(lens, ctypes.c_void_p),
+                        int(num_ctas), int(unit_keys), ctypes.cast(buf, ctypes.c_void_p), n)
+    if m != n:
+        raise LaError(LA_ERR_INVALID_ARG_CODE, "la_pbd_plan")
+    return [tuple(buf[6 * i: 6 * i + 6]) for i in range(n)]

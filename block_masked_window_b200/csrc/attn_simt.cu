@@ -322,6 +322,7 @@ cudaError_t occupancy_rpt(int B, int* ctas) {
 }  // namespace
 
 int simt_rows_per_thread(int R) { return (R + 15) / 16; }
+int simt_tile_keys() { return kTile; }
 
 size_t simt_smem_bytes(int R, int B) {
   return simt_layout(simt_rows_per_thread(R), B, nullptr, nullptr);

@@ -806,7 +806,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 }
 
 int tc_ctas_per_sm() { return 1; }
-int tc_min_chunk() { return kNT; }
+int tc_tile_keys() { return kNT; }
 
 static int tc_nq(int R) { return round_up(R, 16); }
 

@@ -26,18 +26,18 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
   const int b = s / p.Hkv, h = s - b * p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * kCombineRows + warp;
-  const int n = p.pre_g[b + 1] - p.pre_g[b];
+  const int u = p.pre_g[b + 1] - p.pre_g[b];   // plan units of the sequence
   if (r >= p.R) return;
   __nv_bfloat16* dst = p.out + out_row_offset(p, b, h, r);
-  if (n == 0) {
+  if (u == 0) {
     reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
     if (lane == 0 && r == 0 && h == 0) atomicOr(&p.hdr->err, kErrSeqOverflow);
     return;
   }
   const long long T = (long long)p.Hkv * p.pre_g[p.B];
   const long long C = plan_chunk(p, T);
-  const long long off = (long long)p.Hkv * p.pre_g[b] + (long long)h * n;
-  const int c0 = (int)(off / C), c1 = (int)((off + n - 1) / C);
+  const long long off = (long long)p.Hkv * p.pre_g[b] + (long long)h * u;
+  const int c0 = (int)(off / C), c1 = (int)((off + u - 1) / C);
   if (c0 == c1) return;
   const int ns = c1 - c0 + 1;
   const size_t stride = slot_floats(p.rows_pad);

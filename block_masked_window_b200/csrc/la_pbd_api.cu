@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 #include <mutex>
 
 #include "la_pbd.h"
@@ -85,11 +86,11 @@ la_status fill_problem(const la_pbd_cfg* cfg, int32_t W, Problem* p) {
   return LA_OK;
 }
 
-// Grid size: the resident capacity, but no more CTAs than the largest possible key stream
-// (every sequence at full capacity) can keep busy at c_min keys each.
+// Grid size: the resident capacity, but no more CTAs than the largest possible unit stream
+// (every sequence at full capacity) can keep busy at c_min units each.
 int grid_for(const Problem& p, int capacity) {
-  const long long max_tokens = (long long)p.B * p.Hkv * p.S;
-  const long long useful = (max_tokens + p.c_min - 1) / p.c_min;
+  const long long max_units = (long long)p.B * p.Hkv * ((p.S + p.unit - 1) / p.unit);
+  const long long useful = (max_units + p.c_min - 1) / p.c_min;
   return (int)(useful < capacity ? (useful < 1 ? 1 : useful) : capacity);
 }
 
@@ -184,7 +185,8 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
   if (algo == LA_ALGO_TCGEN05) {
     la::TmaMaps maps;
     if (la::make_tma_maps(p, &maps) != cudaSuccess) return LA_ERR_CUDA;
-    p.c_min = la::tc_min_chunk();
+    p.unit = la::tc_tile_keys();
+    p.c_min = 1;
     p.num_ctas = grid_for(p, sms * la::tc_ctas_per_sm());
     e = la::launch_attn_tc(p, &maps.k, &maps.v, &maps.q, &maps.o, s);
   } else {
@@ -193,13 +195,48 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
     if (e != cudaSuccess) return LA_ERR_CUDA;
     if (per_sm < 1) return LA_ERR_UNSUPPORTED;
     if (per_sm > la::kMaxCtasPerSm) per_sm = la::kMaxCtasPerSm;
-    p.c_min = 32;
+    p.unit = la::simt_tile_keys();
+    p.c_min = 1;
     p.num_ctas = grid_for(p, sms * per_sm);
     e = la::launch_attn_simt(p, s);
   }
   if (e != cudaSuccess) return LA_ERR_CUDA;
   e = la::launch_combine(p, s);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t W, const int32_t* seq_lens_host,
+                    int32_t num_ctas, int32_t unit_keys, int32_t* segments,
+                    int32_t max_segments) {
+  la_status st = check_cfg(cfg, W);
+  if (st != LA_OK) return -(int32_t)st;
+  if (!seq_lens_host || num_ctas < 1 || unit_keys < 1 || max_segments < 0 ||
+      (max_segments > 0 && !segments))
+    return -(int32_t)LA_ERR_INVALID_ARG;
+  Problem p;
+  fill_problem(cfg, W, &p);
+  p.seq_lens = seq_lens_host;
+  p.unit = unit_keys;
+  p.c_min = 1;
+  p.num_ctas = num_ctas;
+  std::vector<int> pre(p.B + 1, 0);
+  for (int b = 0; b < p.B; ++b) pre[b + 1] = pre[b] + la::units_of(p, la::visible_len(p, b));
+  const long long T = (long long)p.Hkv * pre[p.B];
+  const long long C = la::plan_chunk(p, T);
+  int32_t count = 0;
+  for (int c = 0; c < num_ctas; ++c) {
+    la::SegmentIter it = la::plan_begin(p, pre.data(), c, C, T);
+    la::Segment sg;
+    while (it.next(p, pre.data(), c, sg)) {
+      if (count < max_segments) {
+        int32_t* r = segments + 6 * (size_t)count;
+        r[0] = c; r[1] = sg.b; r[2] = sg.h; r[3] = sg.j0; r[4] = sg.j1;
+        r[5] = sg.whole ? -1 : sg.slot;
+      }
+      ++count;
+    }
+  }
+  return count;
 }
 
 la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new, const void* v_new,

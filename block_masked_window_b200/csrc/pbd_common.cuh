@@ -1,14 +1,16 @@
 // Shared device-side pieces of the PBD window-attention kernels: constants, the workspace
 // header, the partial-result slot layout and the flattened split-KV work plan.
 //
-// Work plan ("stream-K" over tokens). Sequence s = b * Hkv + h (batch b, KV head h) has
-// N_b = P_b + W visible keys (0 if P_b is invalid). All sequences are laid end to end in one
-// flattened token stream of length T = Hkv * sum_b N_b. CTA c of a grid of G CTAs owns tokens
-// [c*C, (c+1)*C) with C = max(c_min, ceil(T / G)), so every CTA gets the same number of keys
-// whatever the mix of prefix lengths. The part of a sequence that falls in one CTA is a
-// segment; a CTA that holds a whole sequence writes its final output directly, every other
-// segment writes an (m, l, acc) partial to slot c + s, and the combine kernel merges them.
-// Slot c + s is unique because CTAs and sequences advance together along the stream.
+// Work plan ("stream-K" over key tiles). Sequence s = b * Hkv + h (batch b, KV head h) has
+// N_b = P_b + W visible keys (0 if P_b is invalid), cut into U_b = ceil(N_b / unit) units of
+// `unit` keys (the attention kernel's key tile; only a sequence's last unit is partial). All
+// sequences are laid end to end in one flattened stream of T = Hkv * sum_b U_b units. CTA c
+// of a grid of G CTAs owns units [c*C, (c+1)*C) with C = max(c_min, ceil(T / G)), so every
+// CTA gets the same number of whole tiles whatever the mix of prefix lengths, and no tile is
+// ever shared by two CTAs. The part of a sequence that falls in one CTA is a segment; a CTA
+// that holds a whole sequence writes its final output directly, every other segment writes
+// an (m, l, acc) partial to slot c + s, and the combine kernel merges them. Slot c + s is
+// unique because CTAs and sequences advance together along the stream.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -39,13 +41,14 @@ struct Problem {
   __nv_bfloat16* out;           // [B, W, Hq, D]
   float* partials;              // slots, see slot_floats
   WsHeader* hdr;
-  int* pre_g;                   // [B+1] prefix sums of N_b, written by attention CTA 0
+  int* pre_g;                   // [B+1] prefix sums of U_b, written by attention CTA 0
   int B, Hq, Hkv, G, W, S;      // G = Hq / Hkv
   int R;                        // rows per sequence = W * G
   int rows_pad;                 // R rounded up to 16: rows per partial slot
   int mask_mode;                // 0 = PBD window, 1 = causal window
   int num_ctas;                 // grid size of the attention kernel (fixes the chunk size)
-  int c_min;                    // minimum tokens per CTA
+  int unit;                     // keys per plan unit (the attention kernel's key tile)
+  int c_min;                    // minimum units per CTA
   float scale_log2;             // scale * log2(e)
 };
 
@@ -60,13 +63,21 @@ __device__ inline float* slot_ptr(const Problem& p, int slot) {
 }
 
 // Visible keys of sequence b (0 marks an invalid prefix length).
-__device__ inline int visible_len(const Problem& p, int b) {
+// (Host-callable for the plan inspection entry point, where seq_lens is host memory.)
+__host__ __device__ inline int visible_len(const Problem& p, int b) {
+#ifdef __CUDA_ARCH__
   int P = __ldg(p.seq_lens + b);
+#else
+  int P = p.seq_lens[b];
+#endif
   if (P < 0 || (long long)P + p.W > (long long)p.S) return 0;
   return P + p.W;
 }
 
-// Block-wide prefix sum of N_b into pre[0..B] (pre[0] = 0, pre[b+1] = N_0 + ... + N_b).
+// Plan units of sequence b.
+__host__ __device__ inline int units_of(const Problem& p, int n) { return (n + p.unit - 1) / p.unit; }
+
+// Block-wide prefix sum of U_b into pre[0..B] (pre[0] = 0, pre[b+1] = U_0 + ... + U_b).
 // Every thread of the block must call it. `warp_tot` needs one int per warp (<= 32).
 __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
   const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, wid = tid >> 5;
@@ -75,7 +86,7 @@ __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
   if (tid == 0) pre[0] = 0;
   for (int base = 0; base < p.B; base += nthr) {
     int b = base + tid;
-    int x = (b < p.B) ? visible_len(p, b) : 0;
+    int x = (b < p.B) ? units_of(p, visible_len(p, b)) : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -101,13 +112,13 @@ __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
 }
 
 // Chunk size C from the total T (identical in every kernel that uses the plan).
-__device__ inline long long plan_chunk(const Problem& p, long long T) {
+__host__ __device__ inline long long plan_chunk(const Problem& p, long long T) {
   long long c = (T + p.num_ctas - 1) / p.num_ctas;
   return c < p.c_min ? (long long)p.c_min : c;
 }
 
 // Largest b with Hkv * pre[b] <= pos (pos < T). Never returns a zero-length sequence.
-__device__ inline int plan_find_batch(const Problem& p, const int* pre, long long pos) {
+__host__ __device__ inline int plan_find_batch(const Problem& p, const int* pre, long long pos) {
   int lo = 0, hi = p.B - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
@@ -119,7 +130,7 @@ __device__ inline int plan_find_batch(const Problem& p, const int* pre, long lon
 struct Segment {
   int b, h;        // batch, KV head
   int n;           // visible keys of the sequence (N_b)
-  int j0, j1;      // key range of this segment, 0 <= j0 < j1 <= n
+  int j0, j1;      // key range of this segment, 0 <= j0 < j1 <= n, j0 a multiple of unit
   bool whole;      // the segment is the whole sequence
   int slot;        // partial slot (when !whole)
 };
@@ -128,18 +139,21 @@ struct Segment {
 struct SegmentIter {
   long long pos, end;
   int b, h;
-  __device__ bool next(const Problem& p, const int* pre, int c, Segment& sg) {
+  __host__ __device__ bool next(const Problem& p, const int* pre, int c, Segment& sg) {
     while (pos < end) {
-      int n = pre[b + 1] - pre[b];
-      long long s0 = (long long)p.Hkv * pre[b] + (long long)h * n;
-      if (n == 0 || pos >= s0 + n) {  // advance to the next sequence
+      int u = pre[b + 1] - pre[b];
+      long long s0 = (long long)p.Hkv * pre[b] + (long long)h * u;
+      if (u == 0 || pos >= s0 + u) {  // advance to the next sequence
         if (++h == p.Hkv) { h = 0; ++b; }
         continue;
       }
-      long long lo = pos, hi = (end < s0 + n) ? end : s0 + n;
+      long long lo = pos, hi = (end < s0 + u) ? end : s0 + u;
+      const int n = visible_len(p, b);
       sg.b = b; sg.h = h; sg.n = n;
-      sg.j0 = (int)(lo - s0); sg.j1 = (int)(hi - s0);
-      sg.whole = (sg.j0 == 0 && sg.j1 == n);
+      sg.j0 = (int)(lo - s0) * p.unit;
+      const int e = (int)(hi - s0) * p.unit;
+      sg.j1 = e < n ? e : n;
+      sg.whole = (lo == s0 && hi == s0 + u);
       sg.slot = c + b * p.Hkv + h;
       pos = hi;
       return true;
@@ -148,7 +162,7 @@ struct SegmentIter {
   }
 };
 
-__device__ inline SegmentIter plan_begin(const Problem& p, const int* pre, int c, long long C,
+__host__ __device__ inline SegmentIter plan_begin(const Problem& p, const int* pre, int c, long long C,
                                          long long T) {
   SegmentIter it;
   it.pos = (long long)c * C;
@@ -156,10 +170,10 @@ __device__ inline SegmentIter plan_begin(const Problem& p, const int* pre, int c
   it.b = 0; it.h = 0;
   if (it.pos < T) {
     int b = plan_find_batch(p, pre, it.pos);
-    int n = pre[b + 1] - pre[b];
+    int u = pre[b + 1] - pre[b];
     long long off = it.pos - (long long)p.Hkv * pre[b];
     it.b = b;
-    it.h = n > 0 ? (int)(off / n) : 0;
+    it.h = u > 0 ? (int)(off / u) : 0;
     if (it.h >= p.Hkv) it.h = p.Hkv - 1;
   }
   return it;

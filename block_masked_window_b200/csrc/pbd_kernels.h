@@ -31,6 +31,7 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache
 
 // CUDA-core split-KV attention (any R = W * G <= 128).
 int simt_rows_per_thread(int R);
+int simt_tile_keys();
 size_t simt_smem_bytes(int R, int B);
 cudaError_t simt_max_ctas_per_sm(int R, int B, int* ctas);
 cudaError_t launch_attn_simt(const Problem& p, cudaStream_t stream);

@@ -27,7 +27,7 @@ struct TmaMaps {
 };
 
 int tc_ctas_per_sm();
-int tc_min_chunk();
+int tc_tile_keys();
 
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

@@ -152,6 +152,26 @@ la_status la_pbd_attn_static(const la_pbd_cfg* cfg, const void* q, const void* k
                              void* out, void* stream);
 
 /*
+ * Host-side view of the split-KV work plan that la_pbd_attn follows on the device, for
+ * inspection and testing; touches no GPU. The keys [0, P_b + W) of each (sequence b, KV
+ * head h) are cut into units of `unit_keys` keys (the attention kernel's key tile: 128 for
+ * the tcgen05 kernel, 32 for the CUDA-core kernel), all units are laid end to end, and CTA c
+ * of `num_ctas` takes one contiguous run of them; the part of a (b, h) in one CTA is a
+ * segment. Sequences with an invalid prefix length contribute nothing.
+ *   seq_lens_host  host int32 [cfg->batch]
+ *   segments       host int32 [max_segments][6], written in CTA order as
+ *                  {cta, b, h, j0, j1, slot}: keys [j0, j1) of (b, h); slot = -1 when the
+ *                  segment is the whole sequence (its CTA writes the output), else the
+ *                  workspace slot of its partial result
+ * Returns the number of segments (which may exceed max_segments; only the first
+ * max_segments are written), or -la_status on invalid arguments (num_ctas < 1,
+ * unit_keys < 1, a null pointer, an invalid cfg).
+ */
+int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t window_len, const int32_t* seq_lens_host,
+                    int32_t num_ctas, int32_t unit_keys, int32_t* segments,
+                    int32_t max_segments);
+
+/*
  * Synchronise `stream`, read and clear the workspace's sticky device-side error flags.
  * Returns LA_OK, LA_ERR_SEQ_OVERFLOW, LA_ERR_TIMEOUT or LA_ERR_CUDA.
  */
