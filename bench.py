@@ -171,23 +171,34 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
     cfg = bmw.Config.make(B, wl.num_q_heads, wl.num_kv_heads, wi.max_seq, algo=args.algo)
     ws = bmw.Workspace(cfg, W, device=device)
 
-    step_graphs = [capture(torch, lambda d=d: run_step(bmw, cfg, d, seq, W, ws, L)) for d in dev]
+    # One graph replay runs `inner` consecutive steps, each on the next copy in the rotation
+    # (so every call still reads its inputs from HBM), so that workloads of a single layer
+    # call are timed back to back like the 36 layer calls of a decode step, not one call per
+    # graph launch.
+    inner = max(1, math.ceil(8 / L))
+    def seq_of(i):
+        return [dev[(i * inner + j) % copies] for j in range(inner)]
+    ngraphs = copies if inner == 1 else max(1, copies // math.gcd(copies, inner))
+    step_graphs = [capture(torch, lambda ds=seq_of(i): [run_step(bmw, cfg, d, seq, W, ws, L) for d in ds])
+                   for i in range(ngraphs)]
     steps, warmup = args.steps, args.warmup
     clocks = ClockSampler(device.index if device.index is not None else 0)
     clocks.start()
-    ms = time_graphs(torch, step_graphs, steps, warmup, barrier)
+    replays = max(1, math.ceil(steps / inner))
+    ms = time_graphs(torch, step_graphs, replays, warmup, barrier)
     clk = clocks.stop()
     ms = max_over_ranks(ms)
-    ms_per_step = ms / steps
-    value = aggregate_throughput(world, B, steps, ms)
+    ms_per_step = ms / (replays * inner)
+    value = aggregate_throughput(world, B, replays * inner, ms)
 
     # Dominant kernel: the attention call of one layer (attention + split merge), timed alone
     # over the same rotating copies.
-    attn_graphs = [capture(torch, lambda d=d: run_attn_only(bmw, cfg, d, seq, W, ws, L)) for d in dev]
-    reps = max(steps, 20)
+    attn_graphs = [capture(torch, lambda ds=seq_of(i): [run_attn_only(bmw, cfg, d, seq, W, ws, L) for d in ds])
+                   for i in range(ngraphs)]
+    reps = max(1, math.ceil(max(steps, 20) / inner))
     ms_attn = time_graphs(torch, attn_graphs, reps, warmup, barrier)
     ms_attn = max_over_ranks(ms_attn)
-    launch_us = ms_attn * 1e3 / (reps * L)
+    launch_us = ms_attn * 1e3 / (reps * inner * L)
     alg_bytes = workloads.algorithmic_bytes(wi.seq_lens.tolist(), W, wl.num_q_heads,
                                             wl.num_kv_heads, wl.head_dim)
     achieved = alg_bytes / (launch_us * 1e-6) / 1e9
@@ -198,6 +209,9 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
     # End to end through the same API: inputs from pinned host memory, output back to host.
     e2e = None
     if not args.no_e2e:
+        # One step per replay here: each step copies its own inputs in and its output out.
+        one_step = step_graphs if inner == 1 else [
+            capture(torch, lambda d=d: run_step(bmw, cfg, d, seq, W, ws, L)) for d in dev]
         h_in = {n: host[n].pin_memory() for n in ("q", "k_new", "v_new")}
         h_out = torch.empty_like(host["q"]).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in h_in.values())
@@ -206,7 +220,7 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
             d = dev[i % copies]
             for n in h_in:
                 d[n].copy_(h_in[n], non_blocking=True)
-            step_graphs[i % copies].replay()
+            one_step[i % copies].replay()
             h_out.copy_(d["out"], non_blocking=True)
         torch.cuda.synchronize()
         barrier()
@@ -216,7 +230,7 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
             d = dev[i % copies]
             for n in h_in:
                 d[n].copy_(h_in[n], non_blocking=True)
-            step_graphs[i % copies].replay()
+            one_step[i % copies].replay()
             h_out.copy_(d["out"], non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
@@ -225,6 +239,7 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
         e2e = {"value": aggregate_throughput(world, B, steps, ms_e2e), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ms_e2e / steps}
+        del one_step
     del step_graphs, attn_graphs
     return {
         "wi": wi, "ms_per_step": ms_per_step, "value": value, "clocks": clk,

@@ -74,7 +74,9 @@ constexpr int kBarSFull = kBarQEmpty + 2;            // [kSBufs]
 constexpr int kBarPFull = kBarSFull + kSBufs;            // [2]: one per P^T buffer
 constexpr int kBarOFull = kBarPFull + 2;            // [2]: one per P^T buffer
 constexpr int kBarDrain = kBarOFull + 2;
-constexpr int kNumBars = kBarDrain + 1;
+constexpr int kBarKRaw = kBarDrain + 1;              // [kKStages]: K tiles of a fused append
+constexpr int kBarVRaw = kBarKRaw + kKStages;         // [kMaxVStages]: V tiles of a fused append
+constexpr int kNumBars = kBarVRaw + kMaxVStages;
 
 // Shared-memory plan for a given NQ and V ring depth.
 struct TcLayout {
@@ -284,6 +286,65 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 __device__ __forceinline__ int tiles_of(const Segment& sg) { return (sg.j1 - sg.j0 + kNT - 1) / kNT; }
 
+// ---- Fused window append (step a1 inside the attention launch).
+// The window's keys [P, P + W) of a sequence (n = P + W visible keys) come from k_new / v_new.
+// The producer warp of K (or V) loads the rows that fall in key tile [jt, jt + kNT) into
+// registers, writes them to their cache rows (the append), and, once the tile's TMA copy of
+// the cache (whose window rows are stale) has landed, writes them over those rows in shared
+// memory before it releases the tile to the MMA. Each window row lies in exactly one tile of
+// one CTA, so every row is appended once.
+constexpr int kWinRegs = kMaxWindow * 16 / 32;   // 16-byte chunks per lane: W rows x 16 chunks
+
+__device__ __forceinline__ bool tile_window(const Problem& p, const Segment& sg, int jt, int& w0,
+                                            int& w1) {
+  const int P = sg.n - p.W;
+  const int lo = max(jt, P), hi = min(jt + kNT, sg.j1);
+  w0 = lo - P;
+  w1 = hi - P;
+  return lo < hi;
+}
+
+// Lane l holds chunks l, l + 32, ... of the rows [w0, w1) (16 chunks of 16 bytes per row).
+__device__ __forceinline__ void window_load_append(const Problem& p, const Segment& sg,
+                                                   const __nv_bfloat16* src,
+                                                   __nv_bfloat16* cache, int w0, int w1,
+                                                   int lane, uint4 (&v)[kWinRegs]) {
+  const int P = sg.n - p.W;
+  const int cnt = (w1 - w0) * 16;
+#pragma unroll
+  for (int u = 0; u < kWinRegs; ++u) {
+    const int idx = lane + 32 * u;
+    if (idx < cnt) {
+      const int w = w0 + (idx >> 4), ch = idx & 15;
+      const uint4* s = reinterpret_cast<const uint4*>(
+          src + (((size_t)sg.b * p.W + w) * p.Hkv + sg.h) * kHeadDim) + ch;
+      v[u] = __ldg(s);
+      uint4* d = reinterpret_cast<uint4*>(
+          cache + (((size_t)sg.b * p.Hkv + sg.h) * p.S + (size_t)(P + w)) * kHeadDim) + ch;
+      *d = v[u];
+    }
+  }
+}
+
+// Writes the held rows into the tile at `tile` (two 64-channel halves, 128-byte swizzle:
+// 16-byte chunk c of row r of a half sits at r * 128 + ((c ^ (r & 7)) * 16)).
+__device__ __forceinline__ void window_patch(uint32_t tile, const Problem& p, const Segment& sg,
+                                             int jt, int w0, int w1, int lane,
+                                             const uint4 (&v)[kWinRegs]) {
+  const int P = sg.n - p.W;
+  const int cnt = (w1 - w0) * 16;
+#pragma unroll
+  for (int u = 0; u < kWinRegs; ++u) {
+    const int idx = lane + 32 * u;
+    if (idx < cnt) {
+      const int r = P + w0 + (idx >> 4) - jt, ch = idx & 15;
+      const uint32_t a = tile + (uint32_t)((ch >> 3) * kHalfBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[u].x), "r"(v[u].y),
+                   "r"(v[u].z), "r"(v[u].w));
+    }
+  }
+}
+
 }  // namespace
 
 template <int NQ, bool CAUSAL>
@@ -349,6 +410,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     mbar_init(bar(kBarOFull + 0), 1);
     mbar_init(bar(kBarOFull + 1), 1);
     mbar_init(bar(kBarDrain), 1);
+    for (int s = 0; s < kKStages; ++s) mbar_init(bar(kBarKRaw + s), 1);
+    for (int s = 0; s < kMaxVStages; ++s) mbar_init(bar(kBarVRaw + s), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -376,32 +439,68 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer: Q, K
-    if (lane == 0) {
-      SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
-      Segment sg;
-      int g = 0, nseg = 0;
-      bool ok = true;
-      while (ok && it.next(p, pre, blockIdx.x, sg)) {
+    // Lane 0 issues the copies; the whole warp moves the window rows of a fused append.
+    SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
+    Segment sg;
+    int g = 0, nseg = 0;
+    uint32_t raw_par = 0;   // phase parity of each stage's fused-append barrier
+    bool ok = true;
+    while (ok && it.next(p, pre, blockIdx.x, sg)) {
+      if (lane == 0) {
         const int qs = nseg % qbufs, qu = nseg / qbufs;
-        if (qu > 0 && !mbar_wait(bar(kBarQEmpty + qs), (qu - 1) & 1, ctl)) { ok = false; break; }
-        const uint32_t dq = sQ + qs * 2 * kQHalf;
-        mbar_expect_tx(bar(kBarQFull + qs), 2u * p.R * 128u);
-        tma_load_3d(dq, &tmq, bar(kBarQFull + qs), 0, sg.h * p.G, sg.b * p.W);
-        tma_load_3d(dq + kQHalf, &tmq, bar(kBarQFull + qs), 64, sg.h * p.G, sg.b * p.W);
-        const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
-        const int nt = tiles_of(sg);
-        for (int t = 0; t < nt; ++t, ++g) {
-          const int row = row0 + t * kNT;
-          const int ks = g % kKStages, ku = g / kKStages;
-          if (ku > 0 && !mbar_wait(bar(kBarKEmpty + ks), (ku - 1) & 1, ctl)) { ok = false; break; }
-          const uint32_t dk = sK + ks * kTileBytes;
-          mbar_expect_tx(bar(kBarKFull + ks), (uint32_t)kTileBytes);
-          tma_load_2d(dk, &tmk, bar(kBarKFull + ks), 0, row);
-          tma_load_2d(dk + kHalfBytes, &tmk, bar(kBarKFull + ks), 64, row);
+        if (qu > 0 && !mbar_wait(bar(kBarQEmpty + qs), (qu - 1) & 1, ctl)) {
+          ok = false;
+        } else {
+          const uint32_t dq = sQ + qs * 2 * kQHalf;
+          mbar_expect_tx(bar(kBarQFull + qs), 2u * p.R * 128u);
+          tma_load_3d(dq, &tmq, bar(kBarQFull + qs), 0, sg.h * p.G, sg.b * p.W);
+          tma_load_3d(dq + kQHalf, &tmq, bar(kBarQFull + qs), 64, sg.h * p.G, sg.b * p.W);
         }
-        ++nseg;
       }
-      // Drain: the copies issued last must have landed before shared memory is released.
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
+      const int nt = tiles_of(sg);
+      for (int t = 0; t < nt; ++t, ++g) {
+        const int row = row0 + t * kNT, jt = sg.j0 + t * kNT;
+        const int ks = g % kKStages, ku = g / kKStages;
+        int w0 = 0, w1 = 0;
+        const bool fuse = p.k_new != nullptr && tile_window(p, sg, jt, w0, w1);
+        if (lane == 0) {
+          if (ku > 0 && !mbar_wait(bar(kBarKEmpty + ks), (ku - 1) & 1, ctl)) {
+            ok = false;
+          } else {
+            const uint32_t dk = sK + ks * kTileBytes;
+            const uint32_t fb = bar((fuse ? kBarKRaw : kBarKFull) + ks);
+            mbar_expect_tx(fb, (uint32_t)kTileBytes);
+            tma_load_2d(dk, &tmk, fb, 0, row);
+            tma_load_2d(dk + kHalfBytes, &tmk, fb, 64, row);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (fuse) {
+          // While the tile is in flight: fetch the window rows and append them to the cache.
+          uint4 win[kWinRegs];
+          window_load_append(p, sg, p.k_new, p.kc, w0, w1, lane, win);
+          const uint32_t fb = bar(kBarKRaw + ks);
+          if (lane == 0 && !mbar_wait(fb, (raw_par >> ks) & 1u, ctl)) {
+            mbar_drain(fb, (raw_par >> ks) & 1u, 100000000LL);
+            ok = false;
+          }
+          raw_par ^= 1u << ks;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          window_patch(sK + ks * kTileBytes, p, sg, jt, w0, w1, lane, win);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarKFull + ks));
+        }
+      }
+      ++nseg;
+    }
+    // Drain: the copies issued last must have landed before shared memory is released.
+    if (lane == 0) {
       for (int back = 1; back <= kKStages && g - back >= 0; ++back) {
         const int gg = g - back;
         mbar_drain(bar(kBarKFull + gg % kKStages), (gg / kKStages) & 1, 100000000LL);
@@ -410,24 +509,52 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------------ TMA producer: V
-    if (lane == 0) {
-      SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
-      Segment sg;
-      int g = 0;
-      bool ok = true;
-      while (ok && it.next(p, pre, blockIdx.x, sg)) {
-        const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
-        const int nt = tiles_of(sg);
-        for (int t = 0; t < nt; ++t, ++g) {
-          const int row = row0 + t * kNT;
-          const int vs = g % vstages, vu = g / vstages;
-          if (vu > 0 && !mbar_wait(bar(kBarVEmpty + vs), (vu - 1) & 1, ctl)) { ok = false; break; }
-          const uint32_t dv = sV + vs * kTileBytes;
-          mbar_expect_tx(bar(kBarVFull + vs), (uint32_t)kTileBytes);
-          tma_load_2d(dv, &tmv, bar(kBarVFull + vs), 0, row);
-          tma_load_2d(dv + kHalfBytes, &tmv, bar(kBarVFull + vs), 64, row);
+    SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
+    Segment sg;
+    int g = 0;
+    uint32_t raw_par = 0;
+    bool ok = true;
+    while (ok && it.next(p, pre, blockIdx.x, sg)) {
+      const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
+      const int nt = tiles_of(sg);
+      for (int t = 0; t < nt; ++t, ++g) {
+        const int row = row0 + t * kNT, jt = sg.j0 + t * kNT;
+        const int vs = g % vstages, vu = g / vstages;
+        int w0 = 0, w1 = 0;
+        const bool fuse = p.v_new != nullptr && tile_window(p, sg, jt, w0, w1);
+        if (lane == 0) {
+          if (vu > 0 && !mbar_wait(bar(kBarVEmpty + vs), (vu - 1) & 1, ctl)) {
+            ok = false;
+          } else {
+            const uint32_t dv = sV + vs * kTileBytes;
+            const uint32_t fb = bar((fuse ? kBarVRaw : kBarVFull) + vs);
+            mbar_expect_tx(fb, (uint32_t)kTileBytes);
+            tma_load_2d(dv, &tmv, fb, 0, row);
+            tma_load_2d(dv + kHalfBytes, &tmv, fb, 64, row);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (fuse) {
+          // While the tile is in flight: fetch the window rows and append them to the cache.
+          uint4 win[kWinRegs];
+          window_load_append(p, sg, p.v_new, p.vc, w0, w1, lane, win);
+          const uint32_t fb = bar(kBarVRaw + vs);
+          if (lane == 0 && !mbar_wait(fb, (raw_par >> vs) & 1u, ctl)) {
+            mbar_drain(fb, (raw_par >> vs) & 1u, 100000000LL);
+            ok = false;
+          }
+          raw_par ^= 1u << vs;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          window_patch(sV + vs * kTileBytes, p, sg, jt, w0, w1, lane, win);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarVFull + vs));
         }
       }
+    }
+    if (lane == 0) {
       for (int back = 1; back <= vstages && g - back >= 0; ++back) {
         const int gg = g - back;
         mbar_drain(bar(kBarVFull + gg % vstages), (gg / vstages) & 1, 100000000LL);

@@ -158,13 +158,16 @@ la_status la_kv_append(const la_pbd_cfg* cfg, const void* k_new, const void* v_n
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
-la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
-                      const void* v_cache, const int32_t* seq_lens, int32_t W, void* out,
-                      void* workspace, size_t workspace_bytes, void* stream) {
-  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace,
-                                 workspace_bytes);
-  if (st != LA_OK) return st;
+}  // extern "C"
 
+namespace {
+
+// Attention launch (attention kernel + merge) for validated arguments. With k_new / v_new
+// non-null the caller has chosen the tcgen05 kernel, which then also appends the window
+// (caches written through k_cache / v_cache).
+la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, int32_t W, void* out,
+                      void* workspace, const void* k_new, const void* v_new, void* stream) {
   Problem p;
   fill_problem(cfg, W, &p);
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -182,7 +185,12 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
   const int algo = pick_algo(cfg, p.R);
+  if (k_new && algo != LA_ALGO_TCGEN05) return LA_ERR_INVALID_ARG;
   if (algo == LA_ALGO_TCGEN05) {
+    p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    p.kc = const_cast<__nv_bfloat16*>(p.k);
+    p.vc = const_cast<__nv_bfloat16*>(p.v);
     la::TmaMaps maps;
     if (la::make_tma_maps(p, &maps) != cudaSuccess) return LA_ERR_CUDA;
     p.unit = la::tc_tile_keys();
@@ -203,6 +211,20 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
   if (e != cudaSuccess) return LA_ERR_CUDA;
   e = la::launch_combine(p, s);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, int32_t W, void* out,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, nullptr, nullptr,
+                     stream);
 }
 
 int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t W, const int32_t* seq_lens_host,
@@ -247,9 +269,14 @@ la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new, c
                                  workspace_bytes);
   if (st != LA_OK) return st;
   if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return LA_ERR_INVALID_ARG;
+  // The tcgen05 kernel appends the window itself (one launch less per layer); the CUDA-core
+  // kernel runs after the append kernel.
+  if (pick_algo(cfg, W * (cfg->num_q_heads / cfg->num_kv_heads)) == LA_ALGO_TCGEN05)
+    return attn_launch(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, k_new, v_new,
+                       stream);
   st = la_kv_append(cfg, k_new, v_new, k_cache, v_cache, seq_lens, W, stream);
   if (st != LA_OK) return st;
-  return la_pbd_attn(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, workspace_bytes,
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, nullptr, nullptr,
                      stream);
 }
 

@@ -39,6 +39,12 @@ struct Problem {
   const __nv_bfloat16* v;       // [B, Hkv, S, D]
   const int32_t* seq_lens;      // [B]
   __nv_bfloat16* out;           // [B, W, Hq, D]
+  // Fused window append (tcgen05 kernel only; null otherwise): the window's keys/values are
+  // read from k_new / v_new [B, W, Hkv, D] and written into the caches kc / vc (= k, v).
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* kc;
+  __nv_bfloat16* vc;
   float* partials;              // slots, see slot_floats
   WsHeader* hdr;
   int* pre_g;                   // [B+1] prefix sums of U_b, written by attention CTA 0

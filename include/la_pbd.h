@@ -123,7 +123,14 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                       void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * One whole layer call: la_kv_append followed by la_pbd_attn on the same stream.
+ * One whole layer call: the result of la_kv_append followed by la_pbd_attn on the same
+ * stream (same caches afterwards, same output bits). With the tcgen05 kernel (LA_ALGO_AUTO
+ * with W * Hq/Hkv <= 64, or LA_ALGO_TCGEN05) both run in one launch: the attention kernel
+ * reads the window's keys and values from k_new / v_new and writes them into the caches
+ * itself (the fused append; RK3588 model card, "How it differs from the original", item 1:
+ * the window's rows are placed after the reused prefix, with no rollback). k_new and v_new
+ * must not alias the caches. Validation, errors and the treatment of invalid prefix lengths
+ * (no cache write, zero output rows, sticky flag) are those of the two calls.
  */
 la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new,
                       const void* v_new, void* k_cache, void* v_cache,

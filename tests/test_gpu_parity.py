@@ -183,3 +183,36 @@ def test_kernels_agree():
     b = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=bmw.LA_ALGO_SIMT).double()
     rel = float((a - b).norm() / b.norm())
     assert rel < 2e-3, rel
+
+
+@pytest.mark.parametrize("prefixes,W,Hq,Hkv", [
+    ((1024,), 6, 16, 2), ((0, 1, 121, 122, 123, 250, 4000), 6, 16, 2), ((5, 300), 8, 16, 2),
+    ((7, 129, 1000), 1, 16, 2), ((60, 61), 16, 4, 4),
+])
+def test_fused_step_matches_separate_calls(prefixes, W, Hq, Hkv):
+    """la_pbd_step with the tcgen05 kernel appends the window inside the attention launch: its
+    caches must equal the oracle's append bit for bit and its output must equal that of
+    la_kv_append followed by la_pbd_attn bit for bit (window tiles straddling a tile edge,
+    windows longer than the rest of their tile, an empty prefix)."""
+    wi = workloads.random_case(len(prefixes), prefixes, W, num_q_heads=Hq, num_kv_heads=Hkv,
+                               seed=41)
+    li = wi.layers[0]
+    B = len(prefixes)
+    cfg = bmw.Config.make(B, Hq, Hkv, wi.max_seq, algo=bmw.LA_ALGO_TCGEN05)
+    sl = to_dev(wi.seq_lens)
+    q, kn, vn = to_dev(li.q), to_dev(li.k_new), to_dev(li.v_new)
+    kc1, vc1 = to_dev(li.k_cache), to_dev(li.v_cache)
+    kc2, vc2 = to_dev(li.k_cache), to_dev(li.v_cache)
+    out1, out2 = torch.empty_like(q), torch.empty_like(q)
+    ws = bmw.Workspace(cfg, W)
+    bmw.la_pbd_step(cfg, q, kn, vn, kc1, vc1, sl, W, out1, ws)
+    bmw.la_kv_append(cfg, kn, vn, kc2, vc2, sl, W)
+    bmw.la_pbd_attn(cfg, q, kc2, vc2, sl, W, out2, ws)
+    torch.cuda.synchronize()
+    assert bmw.la_pbd_check(ws) == 0
+    k_ref, v_ref = oracle.kv_append(li.k_cache, li.v_cache, li.k_new, li.v_new, wi.seq_lens)
+    assert np.array_equal(kc1.cpu().double().numpy(), k_ref)
+    assert np.array_equal(vc1.cpu().double().numpy(), v_ref)
+    assert torch.equal(out1, out2)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(out1.cpu(), ref, f"fused step {prefixes} W={W}")
