@@ -286,6 +286,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 __device__ __forceinline__ int tiles_of(const Segment& sg) { return (sg.j1 - sg.j0 + kNT - 1) / kNT; }
 
+// P^T rows 16c..16c+15 of one key (thread): bf16 hi and lo halves, one 16-byte store per
+// group of 8 rows. `prow` addresses this key's 16-byte slot in row group 0 of the hi half;
+// row groups are 2048 bytes apart and the lo half follows the NQ/8 hi groups.
+template <int NQ>
+__device__ __forceinline__ void store_pt16_impl(uint32_t prow, int c, const float (&x)[16]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = x[8 * h + 2 * e], b = x[8 * h + 2 * e + 1];
+      hi[e] = pack_bf16x2(a, b);
+      const float ha = __uint_as_float(hi[e] << 16), hb = __uint_as_float(hi[e] & 0xFFFF0000u);
+      lo[e] = pack_bf16x2(a - ha, b - hb);
+    }
+    const int m = 2 * c + h;
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + m * 2048), "r"(hi[0]),
+                 "r"(hi[1]), "r"(hi[2]), "r"(hi[3]));
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + (NQ / 8 + m) * 2048),
+                 "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]));
+  }
+}
+
 // ---- Fused window append (step a1 inside the attention launch).
 // The window's keys [P, P + W) of a sequence (n = P + W visible keys) come from k_new / v_new.
 // The producer warp of K (or V) loads the rows that fall in key tile [jt, jt + kNT) into
@@ -571,7 +594,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       auto issue_qk = [&](int gg) {
         const uint32_t kb = sK + (gg % kKStages) * kTileBytes;
         const uint32_t d = tmem + kColS + (uint32_t)((gg % kSBufs) * NQ);
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
           const uint32_t ka = kb + (kk >> 2) * kHalfBytes + (kk & 3) * 32;
           const uint32_t qa = sQseg + (kk >> 2) * kQHalf + (kk & 3) * 32;
@@ -580,7 +603,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       };
       auto issue_pv = [&](int gg, bool first) {
         const uint32_t vb = sV + (gg % vstages) * kTileBytes;
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < kNT / 16; ++kk) {
           const uint64_t pdesc = sdesc(sP + (gg & 1) * (NQ * 512) + kk * 256, 128, 2048, 0);
           const uint32_t acc = (first && kk == 0) ? 0u : 1u;
@@ -698,54 +721,65 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const uint32_t s_addr = lane_addr + kColS + (gt % kSBufs) * NQ;
         if (!mbar_wait(bar(kBarSFull + gt % kSBufs), (gt / kSBufs) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
-        float x[NQ];
-#pragma unroll
-        for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
-        tc_wait_ld();
+        // P^T is written as hi/lo row groups, one 16-byte store per 8 rows.
+        const uint32_t prow = sP + (gt & 1) * (NQ * 512) + (uint32_t)((row >> 3) * 128 + (row & 7) * 16);
         // A segment's first tile has no references yet: it always takes the exact-maximum
-        // path below, with the raw scores still in x.
+        // path below.
         bool rescale = true;
         if (t > 0) {
-          // y = score * scale_log2 - reference: the vote asks whether some y exceeds the lazy
-          // threshold, and p = 2^y against the current references. Padding rows (q >= R)
-          // need no mask: their Q rows are zero, so their scores are exactly 0.
+          // The common path (hot, fully unrolled): all NQ scores of this key at once,
+          // p = 2^(score * scale_log2 - reference); the vote asks whether some exponent exceeds
+          // the lazy threshold. Padding rows (q >= R) need no mask: their Q rows are zero, so
+          // their scores are exactly 0.
+          float x[NQ];
+#pragma unroll
+          for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
+          tc_wait_ld();
           const float4* mr4 = reinterpret_cast<const float4*>(rowst + cur * NQ);
           bool exceeds = false;
-          if (CAUSAL || key_ok) {
 #pragma unroll
-            for (int c4 = 0; c4 < NQ / 4; ++c4) {
-              const float4 m4 = mr4[c4];
-              const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
+          for (int c4 = 0; c4 < NQ / 4; ++c4) {
+            const float4 m4 = mr4[c4];
+            const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int q = 4 * c4 + e;
-                const float y = fmaf(x[q], c2, -mq[e]);
-                const bool v = CAUSAL ? (key < lim_q[q]) : true;
-                exceeds |= v && (y > kLazyThreshold);
-                x[q] = v ? fast_exp2(y) : 0.f;
-              }
+            for (int e = 0; e < 4; ++e) {
+              const int q = 4 * c4 + e;
+              const float y = fmaf(x[q], c2, -mq[e]);
+              const bool v = CAUSAL ? (key < lim_q[q]) : key_ok;
+              exceeds |= v && (y > kLazyThreshold);
+              x[q] = v ? fast_exp2(y) : 0.f;
             }
-          } else {
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) x[q] = 0.f;
           }
           // CTA-wide vote: raise the references only if some score is far above them.
           rescale = softmax_bar_or(exceeds);
-          if (rescale) {
+          if (!rescale) {
+            // The product that read this P^T buffer two tiles ago must be done.
+            if (gt > 1) {
+              if (!mbar_wait(bar(kBarOFull + (gt & 1)), ((gt - 2) >> 1) & 1, ctl)) { ok = false; break; }
+              tc_fence_after();
+            }
 #pragma unroll
-            for (int c = 0; c < NQ / 16; ++c) tmem_ld16(s_addr + 16 * c, x + 16 * c);
-            tc_wait_ld();
+            for (int c = 0; c < NQ / 16; ++c)
+              store_pt16_impl<NQ>(prow, c, *reinterpret_cast<const float(*)[16]>(x + 16 * c));
           }
         }
         if (rescale) {
+          // The rare path (always taken on a segment's first tile), 16 rows at a time straight
+          // from TMEM in rolled loops: it runs cold, where instruction fetch rather than
+          // arithmetic sets its speed, so small code wins.
           // Exact tile maxima per row (log2 units): warp reduction, then across the warps.
           float* wm = wmax + (gt & 1) * 4 * NQ;
+#pragma unroll 1
+          for (int c = 0; c < NQ / 16; ++c) {
+            float x[16];
+            tmem_ld16(s_addr + 16 * c, x);
+            tc_wait_ld();
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const bool v = CAUSAL ? (key < lim_q[q]) : key_ok;
-            x[q] = v ? x[q] * c2 : -INFINITY;
-            const float m = warp_max_f32(x[q]);
-            if ((q & 31) == lane) wm[w4 * NQ + q] = m;
+            for (int k = 0; k < 16; ++k) {
+              const bool v = CAUSAL ? (key < lim_q[16 * c + k]) : key_ok;
+              const float m = warp_max_f32(v ? x[k] * c2 : -INFINITY);
+              if (k == (lane & 15) && (lane >> 4) == 0) wm[w4 * NQ + 16 * c + k] = m;
+            }
           }
           softmax_bar();
           // Thread q publishes the new reference of row q and the factor that rescales what
@@ -766,29 +800,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             tc_fence_after();
           }
           softmax_bar();
-          const float4* mn4 = reinterpret_cast<const float4*>(mw);
+#pragma unroll 1
+          for (int c = 0; c < NQ / 16; ++c) {
+            float x[16];
+            tmem_ld16(s_addr + 16 * c, x);
+            tc_wait_ld();
+            const float4* mn4 = reinterpret_cast<const float4*>(mw + 16 * c);
 #pragma unroll
-          for (int c4 = 0; c4 < NQ / 4; ++c4) {
-            const float4 m4 = mn4[c4];
-            const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const float4 m4 = mn4[c4];
+              const float mq[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float safe = (mq[e] == -INFINITY) ? 0.f : mq[e];
-              x[4 * c4 + e] = fast_exp2(x[4 * c4 + e] - safe);
+              for (int e = 0; e < 4; ++e) {
+                const int k = 4 * c4 + e;
+                const bool v = CAUSAL ? (key < lim_q[16 * c + k]) : key_ok;
+                const float safe = (mq[e] == -INFINITY) ? 0.f : mq[e];
+                x[k] = v ? fast_exp2(fmaf(x[k], c2, -safe)) : 0.f;
+              }
             }
-          }
-          if (t > 0) {
-            // O hi, O lo, l hi, l lo columns, 16 rows at a time.
-            const float4* al4 = reinterpret_cast<const float4*>(alpha_s);
-#pragma unroll
-            for (int c = 0; c < NQ / 16; ++c) {
+            store_pt16_impl<NQ>(prow, c, x);
+            if (t > 0) {
+              // O hi, O lo, l hi, l lo columns of these 16 rows.
+              const float4* al4 = reinterpret_cast<const float4*>(alpha_s + 16 * c);
               float al[16];
 #pragma unroll
               for (int e4 = 0; e4 < 4; ++e4) {
-                const float4 a4 = al4[4 * c + e4];
+                const float4 a4 = al4[e4];
                 al[4 * e4] = a4.x; al[4 * e4 + 1] = a4.y; al[4 * e4 + 2] = a4.z; al[4 * e4 + 3] = a4.w;
               }
-#pragma unroll
+#pragma unroll 1
               for (int blk = 0; blk < 4; ++blk) {
                 float o[16];
                 const uint32_t col = kColO + blk * NQ + 16 * c;
@@ -799,33 +839,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 tmem_st16(lane_addr + col, o);
               }
             }
-            tc_wait_st();
           }
+          if (t > 0) tc_wait_st();
           // Nobody reads the old references after the barrier above, and the next writer of
           // this buffer waits at the next tile's vote barrier.
           cur ^= 1;
-        } else if (gt > 1) {
-          // The product that read this P^T buffer two tiles ago must be done.
-          if (!mbar_wait(bar(kBarOFull + (gt & 1)), ((gt - 2) >> 1) & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
-        }
-
-        // P^T as hi/lo row groups (one 16-byte store per 8 rows).
-        const uint32_t prow = sP + (gt & 1) * (NQ * 512) + (uint32_t)((row >> 3) * 128 + (row & 7) * 16);
-#pragma unroll
-        for (int m = 0; m < NQ / 8; ++m) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = x[8 * m + 2 * e], b = x[8 * m + 2 * e + 1];
-            hi[e] = pack_bf16x2(a, b);
-            const float ha = __uint_as_float(hi[e] << 16), hb = __uint_as_float(hi[e] & 0xFFFF0000u);
-            lo[e] = pack_bf16x2(a - ha, b - hb);
-          }
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + m * 2048), "r"(hi[0]),
-                       "r"(hi[1]), "r"(hi[2]), "r"(hi[3]));
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + (NQ / 8 + m) * 2048),
-                       "r"(lo[0]), "r"(lo[1]), "r"(lo[2]), "r"(lo[3]));
         }
         // Rows of the V tile past the segment end hold other data: zero them so 0 * x
         // cannot turn into NaN in the tensor-core product.
@@ -858,7 +876,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       float* slot = sg.whole ? nullptr : slot_ptr(p, sg.slot);
       const uint32_t stg = sP;
       float l_own = 0.f;   // row sum of row q = stid (every lane holds every row's sum)
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < NQ / 16; ++c) {
         float ohi[16], olo[16], lhi[16], llo[16];
         tmem_ld16(lane_addr + kColO + 16 * c, ohi);

@@ -7,9 +7,9 @@
 // and are skipped here. Sequences with an invalid prefix length (no visible keys) get zero
 // rows and raise the sticky overflow flag.
 //
-// One warp per output row (4 rows per 128-thread block): lanes first reduce the row's
-// maxima and sums over the partials, keeping the weights in shared memory, then each lane
-// accumulates 4 of the 128 channels over the partials with independent 16-byte loads.
+// One warp per output row (4 rows per 128-thread block): lane k holds partial k's maximum and
+// sum, the warp reduces them (weights kept in shared memory), and each lane accumulates 4 of
+// the 128 channels over the partials with independent 16-byte loads.
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 
@@ -17,6 +17,7 @@ namespace la {
 
 constexpr int kCombineRows = 4;
 constexpr int kCombineMaxSlots = 1024;   // >= partials of one sequence (<= grid size)
+constexpr int kMerge = 16;               // partials loaded in the first round trip
 
 __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem p) {
   __shared__ float s_w[kCombineRows][kCombineMaxSlots];
@@ -43,44 +44,54 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
   const size_t stride = slot_floats(p.rows_pad);
   const float* base = p.partials + (size_t)(c0 + s) * stride;
 
-  float M = -INFINITY;
-  for (int k = lane; k < ns; k += 32) M = fmaxf(M, base[k * stride + r]);
+  // Latency, not bandwidth, decides this kernel: the partials were just written and sit in
+  // L2. So the first kMerge partial rows are loaded together with the maxima and sums (one
+  // round trip for all of them), and the weights are applied afterwards.
+  const float* acc0 = base + 2 * p.rows_pad + (size_t)r * kHeadDim + 4 * lane;
+  float4 a[kMerge];
+#pragma unroll
+  for (int u = 0; u < kMerge; ++u)
+    if (u < ns) a[u] = *reinterpret_cast<const float4*>(acc0 + (size_t)u * stride);
+  float mk = -INFINITY, lk = 0.f;
+  if (lane < ns) {
+    mk = base[(size_t)lane * stride + r];
+    lk = base[(size_t)lane * stride + p.rows_pad + r];
+  }
+  float M = mk;
+  for (int k = lane + 32; k < ns; k += 32) M = fmaxf(M, base[(size_t)k * stride + r]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float L = 0.f;
-  for (int k = lane; k < ns; k += 32) {
-    const float mk = base[k * stride + r];
-    const float w = (mk == -INFINITY) ? 0.f : fast_exp2(mk - M);
-    s_w[warp][k] = w;
-    L = fmaf(w, base[k * stride + p.rows_pad + r], L);
+  float wk = (mk == -INFINITY) ? 0.f : fast_exp2(mk - M);
+  if (lane < ns) s_w[warp][lane] = wk;
+  float L = wk * lk;
+  for (int k = lane + 32; k < ns; k += 32) {
+    const float m2 = base[(size_t)k * stride + r];
+    const float w2 = (m2 == -INFINITY) ? 0.f : fast_exp2(m2 - M);
+    s_w[warp][k] = w2;
+    L = fmaf(w2, base[(size_t)k * stride + p.rows_pad + r], L);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
   __syncwarp();
 
-  const float* acc0 = base + 2 * p.rows_pad + (size_t)r * kHeadDim + 4 * lane;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int k = 0;
-  for (; k + 4 <= ns; k += 4) {
-    float4 a[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) a[u] = *reinterpret_cast<const float4*>(acc0 + (size_t)(k + u) * stride);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float w = s_w[warp][k + u];
+  for (int u = 0; u < kMerge; ++u) {
+    if (u < ns) {
+      const float w = s_w[warp][u];
       acc.x = fmaf(w, a[u].x, acc.x);
       acc.y = fmaf(w, a[u].y, acc.y);
       acc.z = fmaf(w, a[u].z, acc.z);
       acc.w = fmaf(w, a[u].w, acc.w);
     }
   }
-  for (; k < ns; ++k) {
-    const float4 a = *reinterpret_cast<const float4*>(acc0 + (size_t)k * stride);
+  for (int k = kMerge; k < ns; ++k) {
+    const float4 v = *reinterpret_cast<const float4*>(acc0 + (size_t)k * stride);
     const float w = s_w[warp][k];
-    acc.x = fmaf(w, a.x, acc.x);
-    acc.y = fmaf(w, a.y, acc.y);
-    acc.z = fmaf(w, a.z, acc.z);
-    acc.w = fmaf(w, a.w, acc.w);
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
   }
   const float inv = 1.f / L;
   __nv_bfloat162 o01 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
