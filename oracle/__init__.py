@@ -17,4 +17,7 @@ from .pbd import (  # noqa: F401
     window_attention,
     pbd_step,
     block_prefill_attention,
+    kv_append_varwin,
+    window_attention_varwin,
+    pbd_step_varwin,
 )

@@ -193,6 +193,56 @@ def pbd_step(q, k_cache, v_cache, k_new, v_new, seq_lens, scale: float,
     return window_attention(q, k, v, seq_lens, scale, mask=mask, return_probs=return_probs)
 
 
+# --------------------------------------------------------------------------
+# variable window per sequence (the RKLLM engine's step: the a_b accepted tokens plus
+# 5 <text_mask> tokens, so W_b = a_b + 5 differs between sequences of a batch)
+# --------------------------------------------------------------------------
+def kv_append_varwin(k_cache, v_cache, k_new, v_new, seq_lens, window_lens):
+    """Window rows w < W_b of sequence b go to cache rows P_b + w; k_new, v_new are
+    [B, W_max, Hkv, D] with rows w >= W_b unused. Sequences with P_b < 0, W_b < 1,
+    W_b > W_max or P_b + W_b > S are left untouched."""
+    k = _f64(k_cache).copy()
+    v = _f64(v_cache).copy()
+    kn, vn = _f64(k_new), _f64(v_new)
+    P = np.asarray(_f64(seq_lens), dtype=np.int64)
+    Wb = np.asarray(_f64(window_lens), dtype=np.int64)
+    W_max, S = kn.shape[1], k.shape[2]
+    for b in range(k.shape[0]):
+        w = int(Wb[b])
+        if P[b] < 0 or w < 1 or w > W_max or P[b] + w > S:
+            continue
+        for i in range(w):
+            k[b, :, P[b] + i, :] = kn[b, i]
+            v[b, :, P[b] + i, :] = vn[b, i]
+    return k, v
+
+
+def window_attention_varwin(q, k_cache, v_cache, seq_lens, window_lens, scale: float,
+                            mask: str = "pbd"):
+    """Window attention with a window length W_b per sequence.
+
+    q: [B, W_max, Hq, D]; row i < W_b of sequence b sits at position P_b + i and attends
+    exactly as in ``window_attention`` for a window of W_b rows (every row sees keys
+    [0, P_b + W_b) under the PBD mask). Rows i >= W_b are padding: their output is zero.
+    """
+    qf = _f64(q)
+    P = np.asarray(_f64(seq_lens), dtype=np.int64)
+    Wb = np.asarray(_f64(window_lens), dtype=np.int64)
+    out = np.zeros_like(qf)
+    for b in range(qf.shape[0]):
+        w = int(Wb[b])
+        out[b, :w] = window_attention(qf[b:b + 1, :w], k_cache[b:b + 1], v_cache[b:b + 1],
+                                      np.array([P[b]]), scale, mask=mask)[0]
+    return out
+
+
+def pbd_step_varwin(q, k_cache, v_cache, k_new, v_new, seq_lens, window_lens, scale: float,
+                    mask: str = "pbd"):
+    """One layer call with per-sequence windows: append, then window attention."""
+    k, v = kv_append_varwin(k_cache, v_cache, k_new, v_new, seq_lens, window_lens)
+    return window_attention_varwin(q, k, v, seq_lens, window_lens, scale, mask=mask)
+
+
 def block_prefill_attention(q, k, v, block_ids, scale: float):
     """Block-causal attention over whole sequences (SDLM block mask).
 

@@ -244,10 +244,43 @@ def pin_block_prefill(o):
     np.testing.assert_allclose(out, ref[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
 
 
+def pin_varwin_is_sdpa_blockmask(o):
+    """Per-sequence windows (W_b = accepted tokens + masks, RKLLM engine's step): each
+    sequence's rows i < W_b equal fp64 SDPA over its own full sequence with the brute-force
+    block mask of a W_b-row window; padding rows are zero; the append writes exactly the
+    W_b rows of each sequence at P_b.. and nothing else."""
+    W_max, Hq, Hkv, D = 5, 4, 2, 8
+    prefix, wlens = (4, 0, 9), (1, 5, 3)
+    wi, li = _case(B=3, prefix=prefix, W=W_max, Hq=Hq, Hkv=Hkv, D=D, seed=29)
+    wl = torch.tensor(wlens, dtype=torch.int32)
+    sc = wi.workload.scale
+    k, v = o.kv_append_varwin(li.k_cache, li.v_cache, li.k_new, li.v_new, wi.seq_lens, wl)
+    for mode in ("pbd", "causal"):
+        out = o.pbd_step_varwin(li.q, li.k_cache, li.v_cache, li.k_new, li.v_new, wi.seq_lens,
+                                wl, sc, mask=mode)
+        for b in range(3):
+            P, w = prefix[b], wlens[b]
+            T = P + w
+            # the append, written out
+            kk = li.k_cache[b].double().clone()
+            vv = li.v_cache[b].double().clone()
+            kk[:, P:T] = li.k_new[b, :w].double().permute(1, 0, 2)
+            vv[:, P:T] = li.v_new[b, :w].double().permute(1, 0, 2)
+            assert np.array_equal(k[b], kk.numpy()) and np.array_equal(v[b], vv.numpy())
+            mask = torch.from_numpy(o.block_mask_bruteforce(o.pbd_block_ids(P, w, mode == "causal")))
+            qf = torch.zeros(1, Hq, T, D, dtype=torch.float64)
+            qf[0, :, P:, :] = li.q[b, :w].double().permute(1, 0, 2)
+            ref = F.scaled_dot_product_attention(qf, kk[None, :, :T], vv[None, :, :T],
+                                                 attn_mask=mask, scale=sc, enable_gqa=True)
+            np.testing.assert_allclose(out[b, :w].transpose(1, 0, 2), ref[0, :, P:, :].numpy(),
+                                       rtol=1e-12, atol=1e-12)
+            assert not out[b, w:].any()
+
+
 PINS = [pin_golden_mask, pin_mask_bruteforce, pin_worked_example, pin_w1_is_causal_decode,
         pin_window_is_sdpa_blockmask, pin_gqa_is_sdpa_gqa, pin_invariants,
         pin_window_permutation, pin_causal_window_breaks_permutation, pin_append,
-        pin_block_prefill]
+        pin_block_prefill, pin_varwin_is_sdpa_blockmask]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -294,7 +327,28 @@ def _buggy_mask_all(P, W, S):
     return np.ones((W, S), dtype=bool)
 
 
+_real_varwin = opbd.window_attention_varwin
+
+
+def _buggy_varwin_max_window(q, k_cache, v_cache, seq_lens, window_lens, scale, mask="pbd"):
+    # Every sequence treated as if it had the longest window.
+    wmax = np.full(len(np.asarray(window_lens)), np.asarray(q).shape[1] if hasattr(q, "shape") else 0)
+    return _real_varwin(q, k_cache, v_cache, seq_lens, wmax, scale, mask=mask)
+
+
+_real_append_varwin = opbd.kv_append_varwin
+
+
+def _buggy_append_varwin(k_cache, v_cache, k_new, v_new, seq_lens, window_lens):
+    # All W_max rows appended, padding included.
+    W_max = np.asarray(opbd._f64(k_new)).shape[1]
+    return _real_append_varwin(k_cache, v_cache, k_new, v_new, seq_lens,
+                               np.full(len(np.asarray(seq_lens)), W_max))
+
+
 MISTAKES = {
+    "varwin_uses_max_window": ("window_attention_varwin", _buggy_varwin_max_window),
+    "varwin_appends_padding": ("kv_append_varwin", _buggy_append_varwin),
     "gqa_interleaved": ("kv_head_of", _buggy_interleaved_gqa),
     "visible_off_by_one": ("visible_keys", _buggy_visible),
     "causal_window_mask": ("pbd_window_mask", _buggy_mask_causal),
