@@ -49,6 +49,34 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+def kernel_sources_digest():
+    """SHA-256 over the CUDA sources of the library (order fixed), to tell whether a stored
+    ncu traffic figure was taken on the kernels that run now."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_masked_window_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def stored_traffic(workload):
+    """DRAM bytes per attention call measured by ncu (dram__bytes_read.sum +
+    dram__bytes_write.sum of the attention and merge kernels of one call), from
+    profiles/traffic.json, if it was taken on the current sources and this workload."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f)
+        if d.get("sources_sha256") != kernel_sources_digest():
+            return None
+        e = d["workloads"].get(workload)
+        return None if e is None else float(e["dram_bytes_per_call"])
+    except Exception:
+        return None
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -389,7 +417,7 @@ def main():
             "graph": "CUDA graph per step", "algo": args.algo}),
         "roofline": {"bound": "hbm", "achieved": res["achieved_gbs"], "peak": peak,
                      "unit": "GB/s", "frac": res["achieved_gbs"] / peak,
-                     "peak_kind": peak_kind, "traffic": None,
+                     "peak_kind": peak_kind, "traffic": stored_traffic(wl.name),
                      "kernel": "la_pbd_attn (split-KV attention + merge), one layer",
                      "bytes_per_launch": res["alg_bytes"], "launch_us": res["launch_us"]},
         "gpu_launches": res["launches_per_step"] * args.steps,

@@ -16,7 +16,8 @@ __all__ = [
     "LA_MASK_PBD", "LA_MASK_CAUSAL_WINDOW", "LA_ALGO_AUTO", "LA_ALGO_TCGEN05", "LA_ALGO_SIMT",
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
-    "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "Workspace",
+    "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_attn_varwin",
+    "la_pbd_step_varwin", "Workspace",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -34,7 +35,8 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
 
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
-                    "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan"]
+                    "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan",
+                    "la_pbd_attn_varwin", "la_pbd_step_varwin"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: Optional[ctypes.CDLL] = None
@@ -96,6 +98,10 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_check.argtypes = [vp, vp]
     lib.la_pbd_attn_static.restype = i32
     lib.la_pbd_attn_static.argtypes = [cfgp, vp, vp, vp, vp, i32, vp, vp]
+    lib.la_pbd_attn_varwin.restype = i32
+    lib.la_pbd_attn_varwin.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+    lib.la_pbd_step_varwin.restype = i32
+    lib.la_pbd_step_varwin.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.la_pbd_plan.restype = i32
     lib.la_pbd_plan.argtypes = [cfgp, i32, vp, i32, i32, vp, i32]
     _LIB = lib
@@ -256,3 +262,40 @@ def la_pbd_plan(cfg: Config, window_len: int, seq_lens, num_ctas: int, unit_keys
     if m != n:
         raise LaError(LA_ERR_INVALID_ARG_CODE, "la_pbd_plan")
     return [tuple(buf[6 * i: 6 * i + 6]) for i in range(n)]
+
+
+def la_pbd_attn_varwin(cfg: Config, q, k_cache, v_cache, seq_lens, window_lens, window_max: int,
+                       out, workspace: Workspace, stream=None) -> None:
+    """Window attention with per-sequence window lengths (q, out padded to window_max rows)."""
+    W = int(window_max)
+    q_shape, cache_shape, _ = _shapes(cfg, W)
+    _check_tensor(q, "q", "bf16", q_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check_tensor(window_lens, "window_lens", "i32", (cfg.batch,))
+    _check_tensor(out, "out", "bf16", q_shape)
+    _check(load().la_pbd_attn_varwin(ctypes.byref(cfg), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(seq_lens), _ptr(window_lens), W, _ptr(out),
+                                     workspace.data_ptr(), workspace.nbytes, _stream(stream)),
+           "la_pbd_attn_varwin")
+
+
+def la_pbd_step_varwin(cfg: Config, q, k_new, v_new, k_cache, v_cache, seq_lens, window_lens,
+                       window_max: int, out, workspace: Workspace, stream=None) -> None:
+    """Append rows w < W_b of k_new/v_new, then window attention with per-sequence windows."""
+    W = int(window_max)
+    q_shape, cache_shape, new_shape = _shapes(cfg, W)
+    _check_tensor(q, "q", "bf16", q_shape)
+    _check_tensor(k_new, "k_new", "bf16", new_shape)
+    _check_tensor(v_new, "v_new", "bf16", new_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check_tensor(window_lens, "window_lens", "i32", (cfg.batch,))
+    _check_tensor(out, "out", "bf16", q_shape)
+    _check(load().la_pbd_step_varwin(ctypes.byref(cfg), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                     _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                                     _ptr(window_lens), W, _ptr(out), workspace.data_ptr(),
+                                     workspace.nbytes, _stream(stream)),
+           "la_pbd_step_varwin")

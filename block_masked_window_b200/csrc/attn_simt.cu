@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kThreads) pbd_attn_simt_kernel(Problem p) {
 #pragma unroll
       for (int k = 0; k < RPT; ++k) {
         const int r = rg * RPT + k;
-        const int lim = (r < p.R) ? row_limit(p, sg.n, r) : 0;
+        const int lim = (r < p.R) ? row_limit(p, sg.n, sg.w, r) : 0;
         const int lim_seg = lim < sg.j1 ? lim : sg.j1;
         float x0 = (jt + tl < lim_seg) ? sc[k][0] * p.scale_log2 : -INFINITY;
         float x1 = (jt + tl + 16 < lim_seg) ? sc[k][1] * p.scale_log2 : -INFINITY;
@@ -279,7 +279,8 @@ __global__ void __launch_bounds__(kThreads) pbd_attn_simt_kernel(Problem p) {
       const int r = wid + 8 * k;
       if (r >= p.R) continue;
       if (sg.whole) {
-        const float inv = 1.f / s.l[r];
+        // Padding rows of a shorter window (no visible key, l = 0) are written as zeros.
+        const float inv = (r / p.G < sg.w) ? 1.f / s.l[r] : 0.f;
         __nv_bfloat162 o01 = __floats2bfloat162_rn(acc[k][0] * inv, acc[k][1] * inv);
         __nv_bfloat162 o23 = __floats2bfloat162_rn(acc[k][2] * inv, acc[k][3] * inv);
         uint2 packed;

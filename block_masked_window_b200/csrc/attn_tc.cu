@@ -8,10 +8,10 @@
 // the full-rate M = 128 side:
 //   S^T = K  Q^T   (M = 128 keys,     N = NQ rows,       K = 128 channels) -> TMEM fp32
 //   O^T = V^T P^T  (M = 128 channels, N = 2 NQ (hi, lo), K = 128 keys)     -> TMEM fp32
-//   L   = 1   P^T  (M = 128 copies,   N = 2 NQ (hi, lo), K = 128 keys)     -> TMEM fp32
-// The last product, against a constant all-ones tile, accumulates the softmax row sums next
-// to O, so rescaling, precision and the final normalisation treat O and l identically and no
-// thread has to keep or reduce partial sums.
+// The softmax row sums are not a tensor-core product: softmax thread t (key t of every tile)
+// adds its fp32 p values to NQ partial sums kept in its own TMEM lane, after it has handed
+// the tile's P^T to the MMA, and the 128 lanes are reduced once per segment. So the single
+// MMA-issuing thread issues 16 instructions per tile, not 24.
 // NQ = R rounded up to 16 (48 for the PBD window of 6 rows x 8 grouped heads). P is split
 // into P_hi + P_lo (both bf16, residual ~2^-17 P) so that the bf16 tensor-core product keeps
 // fp32-level accuracy; both halves ride in one N = 2 NQ MMA that reads the V tile once.
@@ -28,8 +28,8 @@
 //   warp 6      TMA producer of the V ring (so neither ring waits on the other)
 //   warp 1      TMEM owner and single-thread MMA issuer (non-blocking: issues whichever of
 //               the next S^T or the next O^T product is ready first)
-//   warps 2..5  softmax: thread t of the 128 reads TMEM lane t, i.e. key t of the S^T tile
-//               and channel t of the O^T accumulator
+//   warps 2..5  softmax: thread t of the 128 reads TMEM lane t, i.e. key t of the S^T tile,
+//               channel t of the O^T accumulator and the row-sum partials of key lane t
 //
 // Shared-memory operand layouts: K, V and Q use the 128-byte swizzle written by TMA (K-major
 // for K and Q, MN-major for V as the A operand of O^T); P^T is written by the softmax
@@ -80,7 +80,7 @@ constexpr int kNumBars = kBarVRaw + kMaxVStages;
 
 // Shared-memory plan for a given NQ and V ring depth.
 struct TcLayout {
-  int k, v, q, p, ones, bar, misc, vote, wmax, lim, mref, alpha, pre, end;
+  int k, v, q, p, bar, misc, vote, wmax, lim, mref, alpha, pre, end;
 };
 __host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, int B) {
   // Operand buffers are 1024-byte multiples from a 1024-aligned base; every small region is
@@ -91,8 +91,7 @@ __host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, in
   L.v = L.k + kKStages * kTileBytes;
   L.q = L.v + vstages * kTileBytes;
   L.p = L.q + qbufs * 2 * nq * 128;         // Q: qbufs buffers x two 64-channel halves
-  L.ones = L.p + 2 * nq * 512;              // P^T: 2 buffers x 2*nq/8 row groups of 2048 B
-  L.bar = L.ones + 128;                     // ones: one 8x8 bf16 core matrix, read with zero strides
+  L.bar = L.p + 2 * nq * 512;               // P^T: 2 buffers x 2*nq/8 row groups of 2048 B
   L.misc = a16(L.bar + kNumBars * 8);       // tmem slot, abort flag
   L.vote = L.misc + 16;                     // (unused slot kept for alignment)
   L.wmax = L.vote + 32;                     // [2][4][nq] floats
@@ -320,7 +319,7 @@ constexpr int kWinRegs = kMaxWindow * 16 / 32;   // 16-byte chunks per lane: W r
 
 __device__ __forceinline__ bool tile_window(const Problem& p, const Segment& sg, int jt, int& w0,
                                             int& w1) {
-  const int P = sg.n - p.W;
+  const int P = sg.n - sg.w;
   const int lo = max(jt, P), hi = min(jt + kNT, sg.j1);
   w0 = lo - P;
   w1 = hi - P;
@@ -332,7 +331,7 @@ __device__ __forceinline__ void window_load_append(const Problem& p, const Segme
                                                    const __nv_bfloat16* src,
                                                    __nv_bfloat16* cache, int w0, int w1,
                                                    int lane, uint4 (&v)[kWinRegs]) {
-  const int P = sg.n - p.W;
+  const int P = sg.n - sg.w;
   const int cnt = (w1 - w0) * 16;
 #pragma unroll
   for (int u = 0; u < kWinRegs; ++u) {
@@ -354,7 +353,7 @@ __device__ __forceinline__ void window_load_append(const Problem& p, const Segme
 __device__ __forceinline__ void window_patch(uint32_t tile, const Problem& p, const Segment& sg,
                                              int jt, int w0, int w1, int lane,
                                              const uint4 (&v)[kWinRegs]) {
-  const int P = sg.n - p.W;
+  const int P = sg.n - sg.w;
   const int cnt = (w1 - w0) * 16;
 #pragma unroll
   for (int u = 0; u < kWinRegs; ++u) {
@@ -379,18 +378,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   constexpr int kQHalf = NQ * 128;                 // bytes of one 64-channel half of Q
   constexpr int kColS = 0;                         // S^T buffers at [0, kSBufs NQ)
   constexpr int kColO = kSBufs * NQ;               // O^T (hi | lo)
-  constexpr int kColL = (kSBufs + 2) * NQ;         // row sums (hi | lo)
-  static_assert((kSBufs + 4) * NQ <= kTmemCols, "TMEM columns");
+  constexpr int kColL = (kSBufs + 2) * NQ;         // row-sum partials of each key lane
+  static_assert((kSBufs + 3) * NQ <= kTmemCols, "TMEM columns");
   constexpr uint32_t kIdescQK = idesc_f16(128, NQ, 0, 0);
   constexpr uint32_t kIdescPV = idesc_f16(128, 2 * NQ, 1, 1);
-  constexpr uint32_t kIdescL = idesc_f16(128, 2 * NQ, 0, 1);
 
   extern __shared__ __align__(1024) char smem_raw[];
   char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int vstages = ring & 0xff, qbufs = ring >> 8;   // V ring depth, Q buffers
   const TcLayout L = tc_layout(NQ, vstages, qbufs, p.B);
   const uint32_t sb = smem_u32(base);
-  const uint32_t sK = sb + L.k, sV = sb + L.v, sQ = sb + L.q, sP = sb + L.p, sOnes = sb + L.ones;
+  const uint32_t sK = sb + L.k, sV = sb + L.v, sQ = sb + L.q, sP = sb + L.p;
   auto bar = [&](int i) { return sb + (uint32_t)L.bar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L.misc + 8);
@@ -412,8 +410,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   // Q rows R..NQ-1 must read as zero: clear both Q buffers once (TMA rewrites rows < R).
   for (int i = tid; i < 4 * kQHalf / 16; i += kThreadsTc)
     reinterpret_cast<uint4*>(base + L.q)[i] = make_uint4(0u, 0u, 0u, 0u);
-  for (int i = tid; i < 128 / 16; i += kThreadsTc)     // bf16 1.0 = 0x3F80
-    reinterpret_cast<uint4*>(base + L.ones)[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
   if (tid == 0) {
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
@@ -594,7 +590,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       auto issue_qk = [&](int gg) {
         const uint32_t kb = sK + (gg % kKStages) * kTileBytes;
         const uint32_t d = tmem + kColS + (uint32_t)((gg % kSBufs) * NQ);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
           const uint32_t ka = kb + (kk >> 2) * kHalfBytes + (kk & 3) * 32;
           const uint32_t qa = sQseg + (kk >> 2) * kQHalf + (kk & 3) * 32;
@@ -603,14 +599,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       };
       auto issue_pv = [&](int gg, bool first) {
         const uint32_t vb = sV + (gg % vstages) * kTileBytes;
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < kNT / 16; ++kk) {
           const uint64_t pdesc = sdesc(sP + (gg & 1) * (NQ * 512) + kk * 256, 128, 2048, 0);
           const uint32_t acc = (first && kk == 0) ? 0u : 1u;
           umma(tmem + kColO, sdesc(vb + kk * 2048, kHalfBytes, 1024, 2), pdesc, kIdescPV, acc);
-          // All-ones A: K-major, no swizzle, every core matrix (8 rows x 16 B) is the same
-          // 128 bytes of ones (leading and stride byte offsets 0).
-          umma(tmem + kColL, sdesc(sOnes, 0, 0, 0), pdesc, kIdescL, acc);
         }
       };
       while (ok && it.next(p, pre, blockIdx.x, sg)) {
@@ -706,7 +699,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     while (ok && it.next(p, pre, blockIdx.x, sg)) {
       const int nt = tiles_of(sg);
       for (int q = stid; q < NQ; q += 128) {
-        if (CAUSAL) lim_s[2 * NQ + q] = (q < p.R) ? min(row_limit(p, sg.n, q), sg.j1) : 0;
+        if (CAUSAL) lim_s[2 * NQ + q] = (q < p.R) ? min(row_limit(p, sg.n, sg.w, q), sg.j1) : 0;
         rowst[q] = -INFINITY;            // no reference yet
       }
       softmax_bar();
@@ -726,6 +719,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         // A segment's first tile has no references yet: it always takes the exact-maximum
         // path below.
         bool rescale = true;
+        bool hot = false;     // p of this tile kept in xs, row sums still to be added
+        float xs[NQ];
         if (t > 0) {
           // The common path (hot, fully unrolled): all NQ scores of this key at once,
           // p = 2^(score * scale_log2 - reference); the vote asks whether some exponent exceeds
@@ -753,6 +748,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           // CTA-wide vote: raise the references only if some score is far above them.
           rescale = softmax_bar_or(exceeds);
           if (!rescale) {
+            hot = true;
             // The product that read this P^T buffer two tiles ago must be done.
             if (gt > 1) {
               if (!mbar_wait(bar(kBarOFull + (gt & 1)), ((gt - 2) >> 1) & 1, ctl)) { ok = false; break; }
@@ -761,6 +757,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
             for (int c = 0; c < NQ / 16; ++c)
               store_pt16_impl<NQ>(prow, c, *reinterpret_cast<const float(*)[16]>(x + 16 * c));
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) xs[q] = x[q];
           }
         }
         if (rescale) {
@@ -819,8 +817,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
               }
             }
             store_pt16_impl<NQ>(prow, c, x);
-            if (t > 0) {
-              // O hi, O lo, l hi, l lo columns of these 16 rows.
+            if (t == 0) {
+              tmem_st16(lane_addr + kColL + 16 * c, x);   // row-sum partials start here
+            } else {
+              // O hi, O lo and the row-sum partials of these 16 rows move to the new
+              // references; this tile's p joins the partials.
               const float4* al4 = reinterpret_cast<const float4*>(alpha_s + 16 * c);
               float al[16];
 #pragma unroll
@@ -829,18 +830,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 al[4 * e4] = a4.x; al[4 * e4 + 1] = a4.y; al[4 * e4 + 2] = a4.z; al[4 * e4 + 3] = a4.w;
               }
 #pragma unroll 1
-              for (int blk = 0; blk < 4; ++blk) {
+              for (int blk = 0; blk < 3; ++blk) {
                 float o[16];
                 const uint32_t col = kColO + blk * NQ + 16 * c;
                 tmem_ld16(lane_addr + col, o);
                 tc_wait_ld();
+                if (blk < 2) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) o[e] *= al[e];
+                  for (int e = 0; e < 16; ++e) o[e] *= al[e];
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) o[e] = fmaf(o[e], al[e], x[e]);
+                }
                 tmem_st16(lane_addr + col, o);
               }
             }
           }
-          if (t > 0) tc_wait_st();
+          tc_wait_st();
           // Nobody reads the old references after the barrier above, and the next writer of
           // this buffer waits at the next tile's vote barrier.
           cur ^= 1;
@@ -862,6 +868,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(bar(kBarPFull + (gt & 1)));
+        if (hot) {
+          // Off the MMA's critical path: this tile's p joins the row-sum partials of this
+          // key lane (the previous tile's partial stores have completed: every tile ends
+          // with a wait on them).
+#pragma unroll
+          for (int c = 0; c < NQ / 16; ++c) {
+            float lp[16];
+            tmem_ld16(lane_addr + kColL + 16 * c, lp);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) lp[e] += xs[16 * c + e];
+            tmem_st16(lane_addr + kColL + 16 * c, lp);
+          }
+          tc_wait_st();
+        }
       }
       if (!ok) break;
       const int glast = g + nt - 1;
@@ -875,44 +896,85 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       // stores while the memory system is saturated by the K/V stream.
       float* slot = sg.whole ? nullptr : slot_ptr(p, sg.slot);
       const uint32_t stg = sP;
-      float l_own = 0.f;   // row sum of row q = stid (every lane holds every row's sum)
+      // Row sums: reduce the 128 key lanes' partials, 16 rows at a time. Within a warp a
+      // butterfly halves the values each lane holds at every step (16 + 8 + 4 + 2 + 1
+      // shuffles leave lane l with the warp's sum of row l & 15); the four warps' sums meet in
+      // shared memory.
+      float* lsum = wmax;              // [NQ] row sums of this segment
+      float* wsum = wmax + NQ;         // [4][NQ] per-warp sums
 #pragma unroll 1
       for (int c = 0; c < NQ / 16; ++c) {
-        float ohi[16], olo[16], lhi[16], llo[16];
-        tmem_ld16(lane_addr + kColO + 16 * c, ohi);
-        tmem_ld16(lane_addr + kColO + NQ + 16 * c, olo);
-        tmem_ld16(lane_addr + kColL + 16 * c, lhi);
-        tmem_ld16(lane_addr + kColL + NQ + 16 * c, llo);
+        float v[16];
+        tmem_ld16(lane_addr + kColL + 16 * c, v);
         tc_wait_ld();
-        // All 16 values first, then the stores, so the divisions overlap.
-        float res[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float o = ohi[e] + olo[e], l = lhi[e] + llo[e];
-          if (16 * c + e == stid) l_own = l;
-          res[e] = sg.whole ? o / l : o;
+        for (int e = 0; e < 16; ++e) v[e] += __shfl_xor_sync(0xffffffffu, v[e], 16);
+#pragma unroll
+        for (int h = 8; h >= 1; h >>= 1) {
+          const bool upper = (lane & h) != 0;
+#pragma unroll
+          for (int e = 0; e < h; ++e) {
+            const float give = upper ? v[e] : v[e + h];
+            const float keep = upper ? v[e + h] : v[e];
+            v[e] = keep + __shfl_xor_sync(0xffffffffu, give, h);
+          }
         }
-        if (sg.whole) {
+        if (lane < 16) wsum[w4 * NQ + 16 * c + lane] = v[0];
+      }
+      softmax_bar();
+      float* linv = wmax + 5 * NQ;     // [NQ] reciprocals of the row sums
+      if (stid < NQ) {
+        const float l = (wsum[stid] + wsum[NQ + stid]) + (wsum[2 * NQ + stid] + wsum[3 * NQ + stid]);
+        lsum[stid] = l;
+        linv[stid] = 1.f / l;
+      }
+      softmax_bar();
+      if (sg.whole) {
+        const int rows_w = sg.w * p.G;
+#pragma unroll 1
+        for (int c = 0; c < NQ / 16; ++c) {
+          float ohi[16], olo[16];
+          tmem_ld16(lane_addr + kColO + 16 * c, ohi);
+          tmem_ld16(lane_addr + kColO + NQ + 16 * c, olo);
+          tc_wait_ld();
+          const float4* l4 = reinterpret_cast<const float4*>(linv + 16 * c);
+          float res[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 a4 = l4[e4];
+            const float li[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) res[4 * e4 + e] = (ohi[4 * e4 + e] + olo[4 * e4 + e]) * li[e];
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int q = 16 * c + e;
             if (q >= p.R) break;
-            const __nv_bfloat16 v = __float2bfloat16_rn(res[e]);
+            // Padding rows of a shorter window (no visible key) are written as zeros.
+            const __nv_bfloat16 v = __float2bfloat16_rn(q < rows_w ? res[e] : 0.f);
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 2u),
                          "h"(*reinterpret_cast<const unsigned short*>(&v)));
           }
-        } else {
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < NQ / 16; ++c) {
+          float ohi[16], olo[16];
+          tmem_ld16(lane_addr + kColO + 16 * c, ohi);
+          tmem_ld16(lane_addr + kColO + NQ + 16 * c, olo);
+          tc_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int q = 16 * c + e;
             if (q >= p.R) break;
-            asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 4u), "f"(res[e]));
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 4u),
+                         "f"(ohi[e] + olo[e]));
           }
         }
       }
       if (!sg.whole && stid < p.R) {
         slot[stid] = rowst[cur * NQ + stid];
-        slot[p.rows_pad + stid] = l_own;
+        slot[p.rows_pad + stid] = lsum[stid];
       }
       fence_async_smem();
       softmax_bar();
@@ -990,7 +1052,7 @@ cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tma
   const CUtensorMap& v = *static_cast<const CUtensorMap*>(tmap_v);
   const CUtensorMap& q = *static_cast<const CUtensorMap*>(tmap_q);
   const CUtensorMap& o = *static_cast<const CUtensorMap*>(tmap_o);
-  const bool causal = p.mask_mode != 0;
+  const bool causal = row_limits(p);   // per-row key limits
   switch (tc_nq(p.R)) {
     case 16: return causal ? launch_nq<16, true>(p, k, v, q, o, stream) : launch_nq<16, false>(p, k, v, q, o, stream);
     case 32: return causal ? launch_nq<32, true>(p, k, v, q, o, stream) : launch_nq<32, false>(p, k, v, q, o, stream);

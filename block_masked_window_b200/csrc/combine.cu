@@ -30,6 +30,15 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
   const int u = p.pre_g[b + 1] - p.pre_g[b];   // plan units of the sequence
   if (r >= p.R) return;
   __nv_bfloat16* dst = p.out + out_row_offset(p, b, h, r);
+  if (u > 0 && r / p.G >= window_of(p, b)) {
+    // Padding row of a shorter window: written as zeros by whichever kernel owns the
+    // sequence (here if it was split; the attention kernel if it was whole).
+    const long long T0 = (long long)p.Hkv * p.pre_g[p.B];
+    const long long C0 = plan_chunk(p, T0);
+    const long long off0 = (long long)p.Hkv * p.pre_g[b] + (long long)h * u;
+    if (off0 / C0 != (off0 + u - 1) / C0) reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
+    return;
+  }
   if (u == 0) {
     reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
     if (lane == 0 && r == 0 && h == 0) atomicOr(&p.hdr->err, kErrSeqOverflow);

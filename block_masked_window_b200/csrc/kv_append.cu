@@ -11,8 +11,8 @@ namespace la {
 
 __global__ void __launch_bounds__(256) kv_append_kernel(
     const uint4* __restrict__ k_new, const uint4* __restrict__ v_new, uint4* __restrict__ k_cache,
-    uint4* __restrict__ v_cache, const int32_t* __restrict__ seq_lens, int B, int W, int Hkv,
-    int S) {
+    uint4* __restrict__ v_cache, const int32_t* __restrict__ seq_lens,
+    const int32_t* __restrict__ window_lens, int B, int W, int Hkv, int S) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -23,7 +23,9 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
   const int w = (int)((row / Hkv) % W);
   const int b = (int)(row / ((long long)Hkv * W));
   const int P = __ldg(seq_lens + b);
-  if (P < 0 || (long long)P + W > S) return;  // flagged by the attention kernels
+  const int wb = window_lens ? __ldg(window_lens + b) : W;   // this sequence's window
+  if (P < 0 || wb < 1 || wb > W || (long long)P + wb > S) return;  // flagged by the attention kernels
+  if (w >= wb) return;                         // padding row of a shorter window
   constexpr int kVec = kHeadDim * 2 / 16;      // 16 vectors of 16 bytes per row
   const int c = lane & (kVec - 1);
   const size_t src = (size_t)row * kVec + c;   // [B, W, Hkv, D] row-major
@@ -36,15 +38,15 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
 }
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
-                             const int32_t* seq_lens, int B, int W, int Hkv, int S,
-                             cudaStream_t stream) {
+                             const int32_t* seq_lens, const int32_t* window_lens, int B,
+                             int W, int Hkv, int S, cudaStream_t stream) {
   const long long rows = (long long)B * W * Hkv;
   const int warps_per_block = 8;
   const unsigned grid = (unsigned)((rows + warps_per_block - 1) / warps_per_block);
   return launch_pdl(kv_append_kernel, dim3(grid), dim3(32 * warps_per_block), 0, stream,
                     static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-                    static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), seq_lens, B, W,
-                    Hkv, S);
+                    static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), seq_lens,
+                    window_lens, B, W, Hkv, S);
 }
 
 }  // namespace la

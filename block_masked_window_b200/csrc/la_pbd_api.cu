@@ -153,7 +153,7 @@ la_status la_kv_append(const la_pbd_cfg* cfg, const void* k_new, const void* v_n
   if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
       !aligned(v_cache, 16) || !aligned(seq_lens, 4))
     return LA_ERR_INVALID_ARG;
-  cudaError_t e = la::launch_kv_append(k_new, v_new, k_cache, v_cache, seq_lens, cfg->batch, W,
+  cudaError_t e = la::launch_kv_append(k_new, v_new, k_cache, v_cache, seq_lens, nullptr, cfg->batch, W,
                                        cfg->num_kv_heads, cfg->max_seq, (cudaStream_t)stream);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
@@ -166,10 +166,12 @@ namespace {
 // non-null the caller has chosen the tcgen05 kernel, which then also appends the window
 // (caches written through k_cache / v_cache).
 la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
-                      const void* v_cache, const int32_t* seq_lens, int32_t W, void* out,
-                      void* workspace, const void* k_new, const void* v_new, void* stream) {
+                      const void* v_cache, const int32_t* seq_lens,
+                      const int32_t* window_lens, int32_t W, void* out, void* workspace,
+                      const void* k_new, const void* v_new, void* stream) {
   Problem p;
   fill_problem(cfg, W, &p);
+  p.window_lens = window_lens;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k_cache);
   p.v = static_cast<const __nv_bfloat16*>(v_cache);
@@ -223,7 +225,7 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
   la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace,
                                  workspace_bytes);
   if (st != LA_OK) return st;
-  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, nullptr, nullptr,
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, nullptr, W, out, workspace, nullptr, nullptr,
                      stream);
 }
 
@@ -272,12 +274,45 @@ la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new, c
   // The tcgen05 kernel appends the window itself (one launch less per layer); the CUDA-core
   // kernel runs after the append kernel.
   if (pick_algo(cfg, W * (cfg->num_q_heads / cfg->num_kv_heads)) == LA_ALGO_TCGEN05)
-    return attn_launch(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, k_new, v_new,
+    return attn_launch(cfg, q, k_cache, v_cache, seq_lens, nullptr, W, out, workspace, k_new, v_new,
                        stream);
   st = la_kv_append(cfg, k_new, v_new, k_cache, v_cache, seq_lens, W, stream);
   if (st != LA_OK) return st;
-  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace, nullptr, nullptr,
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, nullptr, W, out, workspace, nullptr, nullptr,
                      stream);
+}
+
+la_status la_pbd_attn_varwin(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* seq_lens,
+                             const int32_t* window_lens, int32_t W_max, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W_max, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  if (!window_lens || !aligned(window_lens, 4)) return LA_ERR_INVALID_ARG;
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, window_lens, W_max, out, workspace,
+                     nullptr, nullptr, stream);
+}
+
+la_status la_pbd_step_varwin(const la_pbd_cfg* cfg, const void* q, const void* k_new,
+                             const void* v_new, void* k_cache, void* v_cache,
+                             const int32_t* seq_lens, const int32_t* window_lens,
+                             int32_t W_max, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W_max, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  if (!window_lens || !aligned(window_lens, 4)) return LA_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return LA_ERR_INVALID_ARG;
+  if (pick_algo(cfg, W_max * (cfg->num_q_heads / cfg->num_kv_heads)) == LA_ALGO_TCGEN05)
+    return attn_launch(cfg, q, k_cache, v_cache, seq_lens, window_lens, W_max, out, workspace,
+                       k_new, v_new, stream);
+  cudaError_t e = la::launch_kv_append(k_new, v_new, k_cache, v_cache, seq_lens, window_lens,
+                                       cfg->batch, W_max, cfg->num_kv_heads, cfg->max_seq,
+                                       (cudaStream_t)stream);
+  if (e != cudaSuccess) return LA_ERR_CUDA;
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, window_lens, W_max, out, workspace,
+                     nullptr, nullptr, stream);
 }
 
 la_status la_pbd_check(void* workspace, void* stream) {

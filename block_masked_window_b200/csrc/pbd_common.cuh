@@ -38,6 +38,7 @@ struct Problem {
   const __nv_bfloat16* k;       // [B, Hkv, S, D]
   const __nv_bfloat16* v;       // [B, Hkv, S, D]
   const int32_t* seq_lens;      // [B]
+  const int32_t* window_lens;   // [B] window length W_b <= W of each sequence, or null (all W)
   __nv_bfloat16* out;           // [B, W, Hq, D]
   // Fused window append (tcgen05 kernel only; null otherwise): the window's keys/values are
   // read from k_new / v_new [B, W, Hkv, D] and written into the caches kc / vc (= k, v).
@@ -48,7 +49,7 @@ struct Problem {
   float* partials;              // slots, see slot_floats
   WsHeader* hdr;
   int* pre_g;                   // [B+1] prefix sums of U_b, written by attention CTA 0
-  int B, Hq, Hkv, G, W, S;      // G = Hq / Hkv
+  int B, Hq, Hkv, G, W, S;      // G = Hq / Hkv; W = the (longest) window length
   int R;                        // rows per sequence = W * G
   int rows_pad;                 // R rounded up to 16: rows per partial slot
   int mask_mode;                // 0 = PBD window, 1 = causal window
@@ -68,16 +69,27 @@ __device__ inline float* slot_ptr(const Problem& p, int slot) {
   return p.partials + (size_t)slot * slot_floats(p.rows_pad);
 }
 
-// Visible keys of sequence b (0 marks an invalid prefix length).
-// (Host-callable for the plan inspection entry point, where seq_lens is host memory.)
+// Window length of sequence b (W when all sequences share it).
+// (Host-callable for the plan inspection entry point, where the arrays are host memory.)
+__host__ __device__ inline int window_of(const Problem& p, int b) {
+  if (!p.window_lens) return p.W;
+#ifdef __CUDA_ARCH__
+  return __ldg(p.window_lens + b);
+#else
+  return p.window_lens[b];
+#endif
+}
+
+// Visible keys of sequence b, P_b + W_b (0 marks an invalid prefix or window length).
 __host__ __device__ inline int visible_len(const Problem& p, int b) {
 #ifdef __CUDA_ARCH__
   int P = __ldg(p.seq_lens + b);
 #else
   int P = p.seq_lens[b];
 #endif
-  if (P < 0 || (long long)P + p.W > (long long)p.S) return 0;
-  return P + p.W;
+  const int w = window_of(p, b);
+  if (P < 0 || w < 1 || w > p.W || (long long)P + w > (long long)p.S) return 0;
+  return P + w;
 }
 
 // Plan units of sequence b.
@@ -135,7 +147,8 @@ __host__ __device__ inline int plan_find_batch(const Problem& p, const int* pre,
 
 struct Segment {
   int b, h;        // batch, KV head
-  int n;           // visible keys of the sequence (N_b)
+  int n;           // visible keys of the sequence (N_b = P_b + W_b)
+  int w;           // window length of the sequence (W_b)
   int j0, j1;      // key range of this segment, 0 <= j0 < j1 <= n, j0 a multiple of unit
   bool whole;      // the segment is the whole sequence
   int slot;        // partial slot (when !whole)
@@ -155,7 +168,7 @@ struct SegmentIter {
       }
       long long lo = pos, hi = (end < s0 + u) ? end : s0 + u;
       const int n = visible_len(p, b);
-      sg.b = b; sg.h = h; sg.n = n;
+      sg.b = b; sg.h = h; sg.n = n; sg.w = window_of(p, b);
       sg.j0 = (int)(lo - s0) * p.unit;
       const int e = (int)(hi - s0) * p.unit;
       sg.j1 = e < n ? e : n;
@@ -191,11 +204,19 @@ __device__ inline size_t out_row_offset(const Problem& p, int b, int h, int r) {
   return (((size_t)b * p.W + i) * p.Hq + (size_t)h * p.G + g) * kHeadDim;
 }
 
-// Number of keys visible to window row i in a sequence of n = P + W visible keys.
-__device__ inline int row_limit(const Problem& p, int n, int r) {
+// Number of keys visible to row r (window row i = r / G) of a sequence of n = P + w visible
+// keys with a window of w rows: all n (PBD mask) or P + i + 1 (causal window); rows of the
+// padding (i >= w) see nothing.
+__device__ inline int row_limit(const Problem& p, int n, int w, int r) {
+  const int i = r / p.G;
+  if (i >= w) return 0;
   if (p.mask_mode == 0) return n;
-  int i = r / p.G;
-  return n - p.W + i + 1;
+  return n - w + i + 1;
+}
+
+// Rows need their own key limits: the causal-window mask or per-sequence windows.
+__host__ __device__ inline bool row_limits(const Problem& p) {
+  return p.mask_mode != 0 || p.window_lens != nullptr;
 }
 
 // Programmatic dependent launch. Every kernel of the library is launched so that it may start

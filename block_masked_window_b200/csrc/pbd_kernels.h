@@ -26,8 +26,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
-                             const int32_t* seq_lens, int B, int W, int Hkv, int S,
-                             cudaStream_t stream);
+                             const int32_t* seq_lens, const int32_t* window_lens, int B, int W,
+                             int Hkv, int S, cudaStream_t stream);
 
 // CUDA-core split-KV attention (any R = W * G <= 128).
 int simt_rows_per_thread(int R);

@@ -159,6 +159,35 @@ la_status la_pbd_attn_static(const la_pbd_cfg* cfg, const void* q, const void* k
                              void* out, void* stream);
 
 /*
+ * Window attention with a window length per sequence (the RKLLM engine's step sends each
+ * sequence's accepted tokens plus 5 <text_mask> tokens, so W_b differs within a batch: RK3588
+ * model card, "How it differs from the original", item 1). Same as la_pbd_attn with W =
+ * W_max for the layouts, except:
+ *   window_lens  device int32 [B], 1 <= W_b <= W_max
+ *   q, out       bf16 [B, W_max, Hq, D]: rows i < W_b of sequence b are its window (row i
+ *                at position P_b + i, seeing keys [0, P_b + W_b), or [0, P_b + i] with
+ *                LA_MASK_CAUSAL_WINDOW); rows i >= W_b are padding, never read into the
+ *                result, and written as zeros.
+ * A sequence with P_b < 0, W_b outside [1, W_max] or P_b + W_b > max_seq gets zero rows and
+ * raises the sticky flag (la_pbd_check). workspace: la_pbd_workspace_bytes(cfg, W_max).
+ */
+la_status la_pbd_attn_varwin(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                             const void* v_cache, const int32_t* seq_lens,
+                             const int32_t* window_lens, int32_t window_max, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One layer call with per-sequence windows: rows w < W_b of k_new / v_new (bf16
+ * [B, W_max, Hkv, D]) are appended at cache rows P_b + w (padding rows are not), then
+ * la_pbd_attn_varwin. Fused into one launch with the tcgen05 kernel, as in la_pbd_step.
+ */
+la_status la_pbd_step_varwin(const la_pbd_cfg* cfg, const void* q, const void* k_new,
+                             const void* v_new, void* k_cache, void* v_cache,
+                             const int32_t* seq_lens, const int32_t* window_lens,
+                             int32_t window_max, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
  * Host-side view of the split-KV work plan that la_pbd_attn follows on the device, for
  * inspection and testing; touches no GPU. The keys [0, P_b + W) of each (sequence b, KV
  * head h) are cut into units of `unit_keys` keys (the attention kernel's key tile: 128 for
