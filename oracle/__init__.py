@@ -17,6 +17,7 @@ from .pbd import (  # noqa: F401
     window_attention,
     pbd_step,
     block_prefill_attention,
+    block_prefill_row,
     kv_append_varwin,
     window_attention_varwin,
     pbd_step_varwin,

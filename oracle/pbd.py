@@ -264,3 +264,21 @@ def block_prefill_attention(q, k, v, block_ids, scale: float):
         e = np.where(M, np.exp(s), 0.0)
         out[:, h, :] = (e / e.sum(axis=1, keepdims=True)) @ vf[:, g, :]
     return out
+
+
+def block_prefill_row(q_row, k, v, i: int, block_ids, scale: float):
+    """Output of query row i alone (all heads) under the block-causal mask of
+    ``block_prefill_attention``: the same definition evaluated for one row, so that long
+    sequences can be checked at sampled rows. q_row: [Hq, D]; k, v: [T, Hkv, D]."""
+    qf, kf, vf = _f64(q_row), _f64(k), _f64(v)
+    Hq, D = qf.shape
+    T, Hkv = kf.shape[0], kf.shape[1]
+    ids = np.asarray(block_ids)
+    allowed = (np.arange(T) <= i) | (ids == ids[i])
+    out = np.zeros((Hq, D), dtype=np.float64)
+    for h in range(Hq):
+        g = kv_head_of(h, Hq, Hkv)
+        s = scale * (kf[allowed, g, :] @ qf[h])
+        e = np.exp(s - s.max())
+        out[h] = (e / e.sum()) @ vf[allowed, g, :]
+    return out

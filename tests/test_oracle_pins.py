@@ -242,6 +242,10 @@ def pin_block_prefill(o):
                                          v.permute(1, 0, 2)[None], attn_mask=mask, scale=0.3,
                                          enable_gqa=True)
     np.testing.assert_allclose(out, ref[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+    # the single-row form, row by row, against the same SDPA reference
+    for i in range(T):
+        row = o.block_prefill_row(q[i], k, v, i, ids, 0.3)
+        np.testing.assert_allclose(row, ref[0, :, i, :].numpy(), rtol=1e-12, atol=1e-12)
 
 
 def pin_varwin_is_sdpa_blockmask(o):

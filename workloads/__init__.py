@@ -214,3 +214,35 @@ def append_bytes(batch: int, window: int, num_kv_heads: int = NUM_KV_HEADS,
                  head_dim: int = HEAD_DIM) -> int:
     """Bytes of one window append: new K and V rows read once and written once."""
     return 2 * 2 * batch * window * num_kv_heads * head_dim * 2
+
+
+@dataclasses.dataclass
+class PrefillInputs:
+    q: torch.Tensor          # bf16 [B, T, Hq, D]
+    k_cache: torch.Tensor    # bf16 [B, Hkv, S, D], rows [0, T_b) hold sequence b
+    v_cache: torch.Tensor    # bf16 [B, Hkv, S, D]
+    seq_lens: torch.Tensor   # int32 [B] = T_b
+    scale: float
+
+
+def prefill_case(lens, num_q_heads: int = NUM_Q_HEADS, num_kv_heads: int = NUM_KV_HEADS,
+                 head_dim: int = HEAD_DIM, seed: int = 1234, t_max: Optional[int] = None,
+                 max_seq: Optional[int] = None, stale_fill: Optional[float] = None) -> PrefillInputs:
+    """Seeded inputs of a block-causal prefill: N(0,1) fp32 draws rounded to bf16, drawn in
+    the order K cache, V cache, Q. ``stale_fill`` overwrites cache rows at and beyond T_b and
+    q rows at and beyond T_b (padding) so that a read outside the valid range shows."""
+    gen = torch.Generator().manual_seed(seed)
+    lens = [int(x) for x in lens]
+    B = len(lens)
+    T = t_max if t_max is not None else max(1, max(lens))
+    S = max_seq if max_seq is not None else _round_up(T, 8)
+    k = torch.randn(B, num_kv_heads, S, head_dim, generator=gen).to(torch.bfloat16)
+    v = torch.randn(B, num_kv_heads, S, head_dim, generator=gen).to(torch.bfloat16)
+    q = torch.randn(B, T, num_q_heads, head_dim, generator=gen).to(torch.bfloat16)
+    if stale_fill is not None:
+        for b, n in enumerate(lens):
+            k[b, :, n:] = stale_fill
+            v[b, :, n:] = stale_fill
+            q[b, n:] = stale_fill
+    return PrefillInputs(q, k, v, torch.tensor(lens, dtype=torch.int32),
+                         1.0 / math.sqrt(head_dim))
