@@ -197,6 +197,8 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
     copies = max(2, min(args.max_copies, math.ceil(2.5 * l2 / max(per_copy, 1))))
     host, dev, seq, L = build_device_inputs(wi, copies, device)
     cfg = bmw.Config.make(B, wl.num_q_heads, wl.num_kv_heads, wi.max_seq, algo=args.algo)
+    R = W * (wl.num_q_heads // wl.num_kv_heads)
+    uses_tc = args.algo == 1 or (args.algo == 0 and R <= 64)
     ws = bmw.Workspace(cfg, W, device=device)
 
     # One graph replay runs `inner` consecutive steps, each on the next copy in the rotation
@@ -273,8 +275,43 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
         "wi": wi, "ms_per_step": ms_per_step, "value": value, "clocks": clk,
         "launch_us": launch_us, "alg_bytes": alg_bytes, "achieved_gbs": achieved,
         "step_bytes": step_bytes, "copies": copies, "e2e": e2e, "layers": L,
-        "launches_per_step": L * 3,
+        # per layer: attention (with the append fused in on the tcgen05 path) + merge; the
+        # CUDA-core path runs the append kernel too
+        "launches_per_step": L * (2 if uses_tc else 3),
     }
+
+
+def measure_prefill(args, device, bmw, torch, barrier, max_over_ranks, T=16384, bs=6):
+    """Block-causal prefill (the pages' long contexts): one sequence of T tokens, 16 query /
+    2 KV heads, block size 6, timed back to back in a CUDA graph over two copies of the inputs
+    (> L2 together). Algorithmic FLOPs: 4 * D * Hq * sum_i visible(i) (QK^T and PV)."""
+    pi = workloads.prefill_case((T,), seed=71)
+    cfg = bmw.Config.make(1, pi.q.shape[2], pi.k_cache.shape[1], pi.k_cache.shape[2])
+    copies = [{n: getattr(pi, n).to(device) for n in ("q", "k_cache", "v_cache", "seq_lens")}
+              for _ in range(2)]
+    for d in copies:
+        d["out"] = torch.empty_like(d["q"])
+    ws = bmw.Workspace(cfg, 1, device=device)
+    run = lambda d: bmw.la_block_prefill(cfg, d["q"], d["k_cache"], d["v_cache"], d["seq_lens"],  # noqa: E731
+                                          bs, d["out"], ws)
+    graphs = [capture(torch, lambda d=d: run(d)) for d in copies]
+    reps = max(4, min(args.steps, 10))
+    ms = max_over_ranks(time_graphs(torch, graphs, reps, args.warmup, barrier)) / reps
+    if bmw.la_pbd_check(ws) != 0:
+        raise RuntimeError("device-side status not OK after the prefill benchmark")
+    i = torch.arange(T, dtype=torch.float64)
+    visible = torch.minimum(torch.full_like(i, T), (torch.floor(i / bs) + 1) * bs).sum().item()
+    flops = 4.0 * 128 * pi.q.shape[2] * visible
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        peak = 1590.0
+    return {"workload": f"block prefill T={T} bs={bs} 16q/2kv d128", "ms": ms,
+            "tflops": tflops, "bound": "tensor", "peak_tflops": peak,
+            "frac_of_measured_bf16": tflops / peak, "flops_per_call": flops}
 
 
 def dist_helpers(world, device):
@@ -345,6 +382,7 @@ def main():
     ap.add_argument("--max-copies", type=int, default=16)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the block-prefill line")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -400,6 +438,9 @@ def main():
             "frac_of_8tbs": r["achieved_gbs"] / 8000.0,
         })
 
+    prefill = None if args.no_prefill else measure_prefill(args, device, bmw, torch, barrier,
+                                                           max_over_ranks)
+
     if rank != 0:
         if world > 1:
             import torch.distributed as dist
@@ -425,6 +466,7 @@ def main():
         "step_bytes": res["step_bytes"],
         "step_gbs": res["step_bytes"] / (res["ms_per_step"] * 1e-3) / 1e9,
         "sweep": sweep,
+        "prefill": prefill,
     }
     print(json.dumps(line))
     if world > 1:

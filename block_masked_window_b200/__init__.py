@@ -17,7 +17,7 @@ __all__ = [
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
     "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_attn_varwin",
-    "la_pbd_step_varwin", "Workspace",
+    "la_pbd_step_varwin", "la_block_prefill", "Workspace",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -36,7 +36,7 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
                     "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan",
-                    "la_pbd_attn_varwin", "la_pbd_step_varwin"]
+                    "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: Optional[ctypes.CDLL] = None
@@ -102,6 +102,8 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_attn_varwin.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.la_pbd_step_varwin.restype = i32
     lib.la_pbd_step_varwin.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+    lib.la_block_prefill.restype = i32
+    lib.la_block_prefill.argtypes = [cfgp, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp]
     lib.la_pbd_plan.restype = i32
     lib.la_pbd_plan.argtypes = [cfgp, i32, vp, i32, i32, vp, i32]
     _LIB = lib
@@ -299,3 +301,20 @@ def la_pbd_step_varwin(cfg: Config, q, k_new, v_new, k_cache, v_cache, seq_lens,
                                      _ptr(window_lens), W, _ptr(out), workspace.data_ptr(),
                                      workspace.nbytes, _stream(stream)),
            "la_pbd_step_varwin")
+
+
+def la_block_prefill(cfg: Config, q, k_cache, v_cache, seq_lens, block_size: int, out,
+                     workspace: Workspace, stream=None) -> None:
+    """Block-causal prefill attention: q, out [B, T, Hq, D]; caches [B, Hkv, S, D] holding
+    each sequence's keys in rows [0, T_b); seq_lens = T_b."""
+    B, T = int(q.shape[0]), int(q.shape[1])
+    Hq, Hkv, D, S = cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, cfg.max_seq
+    _check_tensor(q, "q", "bf16", (B, T, Hq, D))
+    _check_tensor(k_cache, "k_cache", "bf16", (B, Hkv, S, D))
+    _check_tensor(v_cache, "v_cache", "bf16", (B, Hkv, S, D))
+    _check_tensor(seq_lens, "seq_lens", "i32", (B,))
+    _check_tensor(out, "out", "bf16", (B, T, Hq, D))
+    _check(load().la_block_prefill(ctypes.byref(cfg), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                   _ptr(seq_lens), T, int(block_size), _ptr(out),
+                                   workspace.data_ptr(), workspace.nbytes, _stream(stream)),
+           "la_block_prefill")

@@ -315,6 +315,42 @@ la_status la_pbd_step_varwin(const la_pbd_cfg* cfg, const void* q, const void* k
                      nullptr, nullptr, stream);
 }
 
+la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* seq_lens, int32_t t_max,
+                           int32_t block_size, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  la_status st = check_cfg(cfg, 1);
+  if (st != LA_OK) return st;
+  if (!q || !k_cache || !v_cache || !seq_lens || !out) return LA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(seq_lens, 4))
+    return LA_ERR_INVALID_ARG;
+  if (t_max < 1 || block_size < 1) return LA_ERR_INVALID_ARG;
+  if ((long long)cfg->batch * t_max >= (1LL << 31)) return LA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256)) return LA_ERR_WORKSPACE;
+  if (workspace_bytes < (size_t)la::kHeaderBytes) return LA_ERR_WORKSPACE;
+  la::PrefillProblem p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seq_lens = seq_lens;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.hdr = static_cast<la::WsHeader*>(workspace);
+  p.B = cfg->batch;
+  p.Hq = cfg->num_q_heads;
+  p.Hkv = cfg->num_kv_heads;
+  p.G = cfg->num_q_heads / cfg->num_kv_heads;
+  p.S = cfg->max_seq;
+  p.T = t_max;
+  p.bs = block_size;
+  p.scale_log2 = cfg->scale * 1.4426950408889634f;
+  CUtensorMap mq, mk, mv;
+  if (la::make_prefill_maps(p, &mq, &mk, &mv) != cudaSuccess) return LA_ERR_CUDA;
+  cudaError_t e = la::launch_prefill_tc(p, &mq, &mk, &mv, (cudaStream_t)stream);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
 la_status la_pbd_check(void* workspace, void* stream) {
   if (!workspace || !aligned(workspace, 256)) return LA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;

@@ -59,6 +59,19 @@ struct Problem {
   float scale_log2;             // scale * log2(e)
 };
 
+// Launch parameters of the block-causal prefill kernel.
+struct PrefillProblem {
+  const __nv_bfloat16* q;       // [B, T, Hq, D]
+  const __nv_bfloat16* k;       // [B, Hkv, S, D], rows [0, T_b) hold the sequence
+  const __nv_bfloat16* v;       // [B, Hkv, S, D]
+  const int32_t* seq_lens;      // [B] tokens T_b of each sequence
+  __nv_bfloat16* out;           // [B, T, Hq, D]
+  WsHeader* hdr;
+  int B, Hq, Hkv, G, S, T;      // T = padded token count of q / out
+  int bs;                       // block size of the block mask
+  float scale_log2;
+};
+
 __host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 __host__ __device__ inline size_t slot_floats(int rows_pad) {

@@ -41,6 +41,11 @@ size_t tc_smem_bytes(int R, int B);
 cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tmap_v,
                            const void* tmap_q, const void* tmap_o, cudaStream_t stream);
 
+// tcgen05 + TMA block-causal prefill (one CTA per 128 query rows of a (sequence, head)).
+size_t prefill_smem_bytes();
+cudaError_t launch_prefill_tc(const PrefillProblem& p, const void* tmap_q, const void* tmap_k,
+                              const void* tmap_v, cudaStream_t stream);
+
 // Merge of the per-split partials into the bf16 output.
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream);
 

@@ -1,0 +1,398 @@
+// tcgen05 + TMA block-causal prefill attention for sm_100a.
+//
+// The prefill of a block-diffusion decoder uses a block mask over whole sequences: token i
+// attends key j when j <= i or when both lie in the same block of `block_size` consecutive
+// tokens (SDLM-style block mask; the PBD window is the last block of it). For contiguous
+// blocks this is one key limit per row: row i sees keys [0, min(T, (i / bs + 1) * bs)).
+//
+// One CTA computes 128 query rows of one (sequence, query head) against the keys they may
+// see, flash-attention style, on the tensor cores:
+//   S = Q K^T  (M = 128 query rows, N = 128 keys,     K = 128 channels) -> TMEM fp32, 2 bufs
+//   O += P V   (M = 128 query rows, N = 128 channels, K = 128 keys)     -> TMEM fp32
+// Thread r of the 128 softmax threads owns query row r (TMEM lane r): it reads its scores
+// from TMEM, keeps its running reference maximum and row sum in registers, writes its row of
+// P (bf16) into shared memory in the 128-byte-swizzled K-major layout the MMA reads, and at
+// the end normalises its O row and stores it. The reference maximum is lazy (raised only
+// when a score exceeds it by 2^8); a warp whose lanes raise it rescales their O rows in TMEM
+// after the previous PV product has completed.
+//
+// Roles (224 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 6 TMA for the V
+// ring, warp 1 TMEM owner and MMA issuer, warps 2..5 softmax. Query tiles are scheduled
+// longest first (the last tiles see the most keys). Every wait is bounded (sticky timeout
+// flag, drain, TMEM freed, return).
+#include "pbd_common.cuh"
+#include "pbd_kernels.h"
+#include "tc_util.cuh"
+#include "tma_util.h"
+
+namespace la {
+namespace {
+
+using namespace tc;
+
+constexpr int kBM = 128;                 // query rows per CTA
+constexpr int kBN = 128;                 // keys per tile
+constexpr int kPfThreads = 224;
+constexpr int kPfStages = 2;             // K and V ring depth
+constexpr int kPHalf = 128 * 128;        // one 64-column half of a 128-row bf16 tile (16 KB)
+constexpr int kPTile = 2 * kPHalf;       // 32 KB
+constexpr float kPfLazy = 8.f;           // log2 units
+constexpr int kPfTmemCols = 512;
+constexpr int kColS = 0;                 // S: 2 buffers x 128 columns
+constexpr int kColO = 2 * kBN;           // O: 128 columns
+
+constexpr int kBQFull = 0;
+constexpr int kBKFull = 1;                        // [kPfStages]
+constexpr int kBKEmpty = kBKFull + kPfStages;     // [kPfStages]
+constexpr int kBVFull = kBKEmpty + kPfStages;     // [kPfStages]
+constexpr int kBVEmpty = kBVFull + kPfStages;     // [kPfStages]
+constexpr int kBSFull = kBVEmpty + kPfStages;     // [2]
+constexpr int kBPFull = kBSFull + 2;              // [2], 128 arrivals
+constexpr int kBOFull = kBPFull + 2;              // [2], one per P buffer
+constexpr int kBDrain = kBOFull + 2;
+constexpr int kBNum = kBDrain + 1;
+
+// Shared memory: Q | K ring | V ring | P x 2 | barriers | misc.
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kPTile;
+constexpr int kOffV = kOffK + kPfStages * kPTile;
+constexpr int kOffP = kOffV + kPfStages * kPTile;
+constexpr int kOffBar = kOffP + 2 * kPTile;
+constexpr int kOffMisc = kOffBar + kBNum * 8;
+constexpr int kPfSmem = kOffMisc + 16;
+constexpr size_t kPfSmemAlloc = (size_t)kPfSmem + 1024;   // + alignment slack
+
+}  // namespace
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, PrefillProblem p) {
+  extern __shared__ __align__(1024) char smem_raw[];
+  char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(base);
+  const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV, sP = sb + kOffP;
+  auto bar = [&](int i) { return sb + (uint32_t)kOffBar + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ntiles = (p.T + kBM - 1) / kBM;
+  const int tile = ntiles - 1 - (int)blockIdx.x;   // longest first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / p.G;
+  const int i0 = tile * kBM;
+  Ctl ctl{abort_flag, p.hdr};
+
+  pdl_trigger();
+  if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmq)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+    mbar_init(bar(kBQFull), 1);
+    for (int s = 0; s < kPfStages; ++s) {
+      mbar_init(bar(kBKFull + s), 1);
+      mbar_init(bar(kBKEmpty + s), 1);
+      mbar_init(bar(kBVFull + s), 1);
+      mbar_init(bar(kBVEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBSFull + s), 1);
+      mbar_init(bar(kBPFull + s), 128);
+      mbar_init(bar(kBOFull + s), 1);
+    }
+    mbar_init(bar(kBDrain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kPfTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  pdl_wait();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Tokens of this sequence; an invalid length gives zero rows and the sticky flag.
+  int Tb = __ldg(p.seq_lens + b);
+  if (Tb < 0 || Tb > p.T || Tb > p.S) {
+    if (tid == 0 && h == 0 && tile == ntiles - 1) atomicOr(&p.hdr->err, kErrSeqOverflow);
+    Tb = 0;
+  }
+  const int rows_here = min(kBM, p.T - i0);   // rows of `out` this CTA owns
+  const int ilast = min(i0 + kBM, Tb) - 1;    // last valid query row of the tile
+  const int kmax = (ilast >= i0) ? min(Tb, (ilast / p.bs + 1) * p.bs) : 0;
+  const int nk = (kmax + kBN - 1) / kBN;      // key tiles (0: nothing to compute)
+
+  if (nk > 0 && warp == 0) {
+    // ------------------------------------------------------------------ TMA: Q, K
+    if (lane == 0) {
+      bool ok = true;
+      mbar_expect_tx(bar(kBQFull), (uint32_t)kPTile);
+      tma_load_3d(sQ, &tmq, bar(kBQFull), 0, h, b * p.T + i0);
+      tma_load_3d(sQ + kPHalf, &tmq, bar(kBQFull), 64, h, b * p.T + i0);
+      const int row0 = (b * p.Hkv + hk) * p.S;
+      int t = 0;
+      for (; ok && t < nk; ++t) {
+        const int s = t % kPfStages, u = t / kPfStages;
+        if (u > 0 && !mbar_wait(bar(kBKEmpty + s), (u - 1) & 1, ctl)) { ok = false; break; }
+        mbar_expect_tx(bar(kBKFull + s), (uint32_t)kPTile);
+        tma_load_2d(sK + s * kPTile, &tmk, bar(kBKFull + s), 0, row0 + t * kBN);
+        tma_load_2d(sK + s * kPTile + kPHalf, &tmk, bar(kBKFull + s), 64, row0 + t * kBN);
+      }
+      for (int back = 1; back <= kPfStages && t - back >= 0; ++back) {
+        const int tt = t - back;
+        mbar_drain(bar(kBKFull + tt % kPfStages), (tt / kPfStages) & 1, 100000000LL);
+      }
+      mbar_drain(bar(kBQFull), 0, 100000000LL);
+    }
+  } else if (nk > 0 && warp == 6) {
+    // ------------------------------------------------------------------ TMA: V
+    if (lane == 0) {
+      bool ok = true;
+      const int row0 = (b * p.Hkv + hk) * p.S;
+      int t = 0;
+      for (; ok && t < nk; ++t) {
+        const int s = t % kPfStages, u = t / kPfStages;
+        if (u > 0 && !mbar_wait(bar(kBVEmpty + s), (u - 1) & 1, ctl)) { ok = false; break; }
+        mbar_expect_tx(bar(kBVFull + s), (uint32_t)kPTile);
+        tma_load_2d(sV + s * kPTile, &tmv, bar(kBVFull + s), 0, row0 + t * kBN);
+        tma_load_2d(sV + s * kPTile + kPHalf, &tmv, bar(kBVFull + s), 64, row0 + t * kBN);
+      }
+      for (int back = 1; back <= kPfStages && t - back >= 0; ++back) {
+        const int tt = t - back;
+        mbar_drain(bar(kBVFull + tt % kPfStages), (tt / kPfStages) & 1, 100000000LL);
+      }
+    }
+  } else if (nk > 0 && warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_f16(128, kBN, 0, 0);     // Q K-major, K K-major
+      constexpr uint32_t kIdO = idesc_f16(128, 128, 0, 1);     // P K-major, V MN-major
+      bool ok = mbar_wait(bar(kBQFull), 0, ctl);
+      tc_fence_after();
+      int nqk = 0, npv = 0;
+      long long t_prog = now_ns();
+      uint32_t spins = 0;
+      while (ok && npv < nk) {
+        bool prog = false;
+        if (nqk < nk && nqk <= npv + 1) {
+          const int s = nqk % kPfStages;
+          if (mbar_test(bar(kBKFull + s), (nqk / kPfStages) & 1)) {
+            tc_fence_after();
+            const uint32_t d = tmem + kColS + (uint32_t)((nqk & 1) * kBN);
+            const uint32_t kb = sK + s * kPTile;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t qa = sQ + (kk >> 2) * kPHalf + (kk & 3) * 32;
+              const uint32_t ka = kb + (kk >> 2) * kPHalf + (kk & 3) * 32;
+              umma(d, sdesc(qa, 16, 1024, 2), sdesc(ka, 16, 1024, 2), kIdS, kk > 0);
+            }
+            umma_commit(bar(kBSFull + (nqk & 1)));
+            umma_commit(bar(kBKEmpty + s));
+            ++nqk;
+            prog = true;
+          }
+        }
+        if (npv < nqk) {
+          const int s = npv % kPfStages;
+          if (mbar_test(bar(kBPFull + (npv & 1)), (npv >> 1) & 1) &&
+              mbar_test(bar(kBVFull + s), (npv / kPfStages) & 1)) {
+            tc_fence_after();
+            const uint32_t pb = sP + (npv & 1) * kPTile;
+            const uint32_t vb = sV + s * kPTile;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t pa = pb + (kk >> 2) * kPHalf + (kk & 3) * 32;
+              umma(tmem + kColO, sdesc(pa, 16, 1024, 2), sdesc(vb + kk * 2048, kPHalf, 1024, 2),
+                   kIdO, (npv > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(bar(kBOFull + (npv & 1)));
+            umma_commit(bar(kBVEmpty + s));
+            ++npv;
+            prog = true;
+          }
+        }
+        if (prog) {
+          spins = 0;
+          t_prog = now_ns();
+          continue;
+        }
+        __nanosleep(32);
+        if ((++spins & 63u) == 0) {
+          if (*abort_flag) { ok = false; break; }
+          if (now_ns() - t_prog > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(&p.hdr->err, kErrTimeout);
+            ok = false;
+            break;
+          }
+        }
+      }
+      umma_commit(bar(kBDrain));
+      mbar_drain(bar(kBDrain), 0, 100000000LL);
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------------------------------------ softmax warps
+    const int sub = warp & 3;
+    const int r = 32 * sub + lane;                 // query row of this thread (TMEM lane)
+    const int i = i0 + r;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * sub) << 16);
+    const int lim = (i < Tb) ? min(Tb, (i / p.bs + 1) * p.bs) : 0;   // keys [0, lim)
+    const float c2 = p.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < nk; ++t) {
+      const int j0 = t * kBN;
+      const uint32_t s_addr = lane_addr + kColS + (uint32_t)((t & 1) * kBN);
+      // (Every lane waits on the same barrier; the vote keeps the error path warp-uniform.)
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBSFull + (t & 1)), (t >> 1) & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+      // Pass 1: the tile's maximum over this row's visible keys (log2 units).
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 16; ++c) {
+        float x[16];
+        tmem_ld16(s_addr + 16 * c, x);
+        tc_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (j0 + 16 * c + e < lim) mt = fmaxf(mt, x[e] * c2);
+      }
+      // Lazy reference: raise it only when a score exceeds it by more than 2^8.
+      const bool raise = mt > m_ref + kPfLazy || (m_ref == -INFINITY && mt > -INFINITY);
+      float alpha = 1.f;
+      if (raise) {
+        alpha = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mt);
+        l *= alpha;
+        m_ref = mt;
+      }
+      // Rows whose reference moved rescale their O row (warp-uniform TMEM access), once
+      // the previous PV product is complete.
+      if (t > 0 && __any_sync(0xffffffffu, raise)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl))) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 128 / 16; ++c) {
+          float o[16];
+          tmem_ld16(lane_addr + kColO + 16 * c, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] *= alpha;
+          tmem_st16(lane_addr + kColO + 16 * c, o);
+        }
+        tc_wait_st();
+      }
+      // The P buffer of this tile was last read by the PV product two tiles ago.
+      if (t > 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + (t & 1)), ((t - 2) >> 1) & 1, ctl))) { ok = false; break; }
+        tc_fence_after();
+      }
+      // Pass 2: p = 2^(x c2 - m_ref) on visible keys, bf16 into the swizzled K-major P tile.
+      const uint32_t prow = sP + (t & 1) * kPTile + (uint32_t)r * 128u;
+      const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 16; ++c) {
+        float x[16];
+        tmem_ld16(s_addr + 16 * c, x);
+        tc_wait_ld();
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float a = (j0 + 16 * c + e < lim) ? fast_exp2(fmaf(x[e], c2, -mref)) : 0.f;
+          const float bq = (j0 + 16 * c + e + 1 < lim) ? fast_exp2(fmaf(x[e + 1], c2, -mref)) : 0.f;
+          l += a + bq;
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bq);
+          pk[e >> 1] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int k8 = 2 * c + hh;                   // 8-key chunk 0..15
+          const uint32_t a = prow + (uint32_t)((k8 >> 3) * kPHalf + (((k8 & 7) ^ (r & 7)) << 4));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * hh]),
+                       "r"(pk[4 * hh + 1]), "r"(pk[4 * hh + 2]), "r"(pk[4 * hh + 3]));
+        }
+      }
+      // Keys past the visible range in the last tile: zero their V rows so that 0 * x
+      // cannot become NaN in the product (those rows may hold anything).
+      const int valid = min(kBN, kmax - j0);
+      if (valid < kBN) {
+        const int s = t % kPfStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBVFull + s), (t / kPfStages) & 1, ctl))) { ok = false; break; }
+        const uint32_t vbase = sV + s * kPTile;
+        for (int idx = r; idx < (kBN - valid) * 16; idx += 128) {
+          const int rr = valid + (idx >> 4), ch = idx & 15;
+          const uint32_t a = vbase + (ch >> 3) * kPHalf + rr * 128 + (ch & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(0u), "r"(0u),
+                       "r"(0u), "r"(0u));
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(kBPFull + (t & 1)));
+    }
+    // Epilogue: O row / l as bf16, straight to global memory (256 contiguous bytes per row).
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBOFull + ((nk - 1) & 1)), ((nk - 1) >> 1) & 1, ctl));
+    tc_fence_after();
+    __nv_bfloat16* dst = p.out + (((size_t)b * p.T + i) * p.Hq + h) * kHeadDim;
+    const float inv = (ok && i < Tb && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 128 / 16; ++c) {
+      float o[16];
+      if (ok) {   // (warp-uniform)
+        tmem_ld16(lane_addr + kColO + 16 * c, o);
+        tc_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = 0.f;
+      }
+      uint32_t pk[8];
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        __nv_bfloat162 v2 = __floats2bfloat162_rn(o[e] * inv, o[e + 1] * inv);
+        pk[e >> 1] = *reinterpret_cast<uint32_t*>(&v2);
+      }
+      if (r < rows_here) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * c);
+        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+    }
+  }
+  if (nk == 0 && warp >= 2 && warp <= 5) {
+    // No valid row in this tile: the owned rows of `out` are zeros.
+    const int r = 32 * (warp & 3) + lane;
+    if (r < rows_here) {
+      uint4* d4 = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.T + i0 + r) * p.Hq + h) * kHeadDim);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) d4[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPfTmemCols));
+  }
+}
+
+size_t prefill_smem_bytes() { return kPfSmemAlloc; }
+
+cudaError_t launch_prefill_tc(const PrefillProblem& p, const void* tmap_q, const void* tmap_k,
+                              const void* tmap_v, cudaStream_t stream) {
+  const CUtensorMap& q = *static_cast<const CUtensorMap*>(tmap_q);
+  const CUtensorMap& k = *static_cast<const CUtensorMap*>(tmap_k);
+  const CUtensorMap& v = *static_cast<const CUtensorMap*>(tmap_v);
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kPfSmemAlloc);
+  if (e != cudaSuccess) return e;
+  const int ntiles = (p.T + kBM - 1) / kBM;
+  return launch_pdl(prefill_tc_kernel, dim3(ntiles, p.Hq, p.B), dim3(kPfThreads), kPfSmemAlloc,
+                    stream, q, k, v, p);
+}
+
+}  // namespace la

@@ -80,4 +80,36 @@ inline cudaError_t make_tma_maps(const Problem& p, TmaMaps* m) {
   return cudaSuccess;
 }
 
+// Prefill maps: q [B*T rows, Hq, 128] with a box of (64 channels, 1 head, 128 tokens); the K
+// and V caches as for the decode kernel (64 channels x 128 rows), all with the 128-byte swizzle.
+inline cudaError_t make_prefill_maps(const PrefillProblem& p, CUtensorMap* mq, CUtensorMap* mk,
+                                     CUtensorMap* mv) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)p.Hq, (cuuint64_t)p.B * p.T};
+    cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)p.Hq * kHeadDim * 2};
+    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)p.q, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const cuuint64_t rows = (cuuint64_t)p.B * p.Hkv * p.S;
+  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (enc(mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)p.k, dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (enc(mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)p.v, dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
 }  // namespace la

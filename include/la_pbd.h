@@ -188,6 +188,26 @@ la_status la_pbd_step_varwin(const la_pbd_cfg* cfg, const void* q, const void* k
                              size_t workspace_bytes, void* stream);
 
 /*
+ * Block-causal prefill attention (the block mask of block-diffusion decoding over whole
+ * sequences; the PBD window is the last block of it): token i of sequence b attends key j
+ * when j <= i or when both lie in the same block of block_size consecutive tokens, i.e. j <
+ * min(T_b, (i / block_size + 1) * block_size).
+ *   q, out         bf16 [B, t_max, Hq, D] (rows i >= T_b of out are written as zeros)
+ *   k_cache,v_cache bf16 [B, Hkv, S_max, D] with the sequence's keys/values in rows [0, T_b)
+ *   seq_lens       device int32 [B]: T_b, 0 <= T_b <= min(t_max, S_max)
+ *   block_size     >= 1
+ *   workspace      >= 256 bytes (its header, zeroed by la_pbd_workspace_init, receives the
+ *                  sticky flags read by la_pbd_check)
+ * bf16 inputs, fp32 accumulation, probabilities rounded to bf16 for the PV product, bf16 out.
+ * A sequence with T_b outside [0, min(t_max, S_max)] gets zero rows and the sticky flag.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* seq_lens, int32_t t_max,
+                           int32_t block_size, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
  * Host-side view of the split-KV work plan that la_pbd_attn follows on the device, for
  * inspection and testing; touches no GPU. The keys [0, P_b + W) of each (sequence b, KV
  * head h) are cut into units of `unit_keys` keys (the attention kernel's key tile: 128 for
