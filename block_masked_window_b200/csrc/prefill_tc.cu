@@ -251,17 +251,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // (Every lane waits on the same barrier; the vote keeps the error path warp-uniform.)
       if (!__all_sync(0xffffffffu, mbar_wait(bar(kBSFull + (t & 1)), (t >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
-      // Pass 1: the tile's maximum over this row's visible keys (log2 units).
-      float mt = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < kBN / 16; ++c) {
-        float x[16];
-        tmem_ld16(s_addr + 16 * c, x);
-        tc_wait_ld();
+      // The row's 128 scores, one TMEM read (4 x 32 columns, one wait).
+      float x[kBN];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (j0 + 16 * c + e < lim) mt = fmaxf(mt, x[e] * c2);
+      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(s_addr + 32 * c, x + 32 * c);
+      tc_wait_ld();
+      // Tiles wholly below this row's limit need no mask (all but the last one or two).
+      const bool full = j0 + kBN <= lim;
+      float mt = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int e = 0; e < kBN; ++e) mt = fmaxf(mt, x[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < kBN; ++e) {
+          if (j0 + e >= lim) x[e] = -INFINITY;
+          mt = fmaxf(mt, x[e]);
+        }
       }
+      mt *= c2;   // log2 units (c2 > 0)
       // Lazy reference: raise it only when a score exceeds it by more than 2^8.
       const bool raise = mt > m_ref + kPfLazy || (m_ref == -INFINITY && mt > -INFINITY);
       float alpha = 1.f;
@@ -291,30 +299,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + (t & 1)), ((t - 2) >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
       }
-      // Pass 2: p = 2^(x c2 - m_ref) on visible keys, bf16 into the swizzled K-major P tile.
+      // p = 2^(x c2 - m_ref) (masked scores are -inf: p = 0), bf16 into the swizzled
+      // K-major P tile, 8 keys per 16-byte store.
       const uint32_t prow = sP + (t & 1) * kPTile + (uint32_t)r * 128u;
       const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
-#pragma unroll 1
-      for (int c = 0; c < kBN / 16; ++c) {
-        float x[16];
-        tmem_ld16(s_addr + 16 * c, x);
-        tc_wait_ld();
-        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const float a = (j0 + 16 * c + e < lim) ? fast_exp2(fmaf(x[e], c2, -mref)) : 0.f;
-          const float bq = (j0 + 16 * c + e + 1 < lim) ? fast_exp2(fmaf(x[e + 1], c2, -mref)) : 0.f;
+      for (int k8 = 0; k8 < kBN / 8; ++k8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          const float a = fast_exp2(fmaf(x[8 * k8 + e], c2, -mref));
+          const float bq = fast_exp2(fmaf(x[8 * k8 + e + 1], c2, -mref));
           l += a + bq;
           __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bq);
           pk[e >> 1] = *reinterpret_cast<uint32_t*>(&v2);
         }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int k8 = 2 * c + hh;                   // 8-key chunk 0..15
-          const uint32_t a = prow + (uint32_t)((k8 >> 3) * kPHalf + (((k8 & 7) ^ (r & 7)) << 4));
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * hh]),
-                       "r"(pk[4 * hh + 1]), "r"(pk[4 * hh + 2]), "r"(pk[4 * hh + 3]));
-        }
+        const uint32_t a = prow + (uint32_t)((k8 >> 3) * kPHalf + (((k8 & 7) ^ (r & 7)) << 4));
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[0]), "r"(pk[1]),
+                     "r"(pk[2]), "r"(pk[3]));
       }
       // Keys past the visible range in the last tile: zero their V rows so that 0 * x
       // cannot become NaN in the product (those rows may hold anything).
