@@ -17,7 +17,8 @@ __all__ = [
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
     "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_attn_varwin",
-    "la_pbd_step_varwin", "la_block_prefill", "Workspace",
+    "la_pbd_step_varwin", "la_block_prefill", "la_pbd_attn_paged", "la_pbd_step_paged",
+    "Workspace",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -36,7 +37,8 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
                     "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan",
-                    "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill"]
+                    "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill",
+                    "la_pbd_attn_paged", "la_pbd_step_paged"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: Optional[ctypes.CDLL] = None
@@ -104,6 +106,11 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_step_varwin.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.la_block_prefill.restype = i32
     lib.la_block_prefill.argtypes = [cfgp, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp]
+    lib.la_pbd_attn_paged.restype = i32
+    lib.la_pbd_attn_paged.argtypes = [cfgp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, sz, vp]
+    lib.la_pbd_step_paged.restype = i32
+    lib.la_pbd_step_paged.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp,
+                                      sz, vp]
     lib.la_pbd_plan.restype = i32
     lib.la_pbd_plan.argtypes = [cfgp, i32, vp, i32, i32, vp, i32]
     _LIB = lib
@@ -318,3 +325,44 @@ def la_block_prefill(cfg: Config, q, k_cache, v_cache, seq_lens, block_size: int
                                    _ptr(seq_lens), T, int(block_size), _ptr(out),
                                    workspace.data_ptr(), workspace.nbytes, _stream(stream)),
            "la_block_prefill")
+
+
+def _check_paged(cfg, q, k_pool, v_pool, block_table, seq_lens, W, out):
+    B, Hq, Hkv, D = cfg.batch, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim
+    _check_tensor(q, "q", "bf16", (B, W, Hq, D))
+    _check_tensor(out, "out", "bf16", (B, W, Hq, D))
+    _check_tensor(k_pool, "k_pool", "bf16")
+    _check_tensor(v_pool, "v_pool", "bf16", tuple(k_pool.shape))
+    if k_pool.dim() != 4 or k_pool.shape[1] != Hkv or k_pool.shape[3] != D:
+        raise ValueError(f"k_pool: expected [num_pages, {Hkv}, page_size, {D}], got {tuple(k_pool.shape)}")
+    _check_tensor(block_table, "block_table", "i32")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table: expected [{B}, pages_per_seq], got {tuple(block_table.shape)}")
+    _check_tensor(seq_lens, "seq_lens", "i32", (B,))
+    return int(k_pool.shape[0]), int(k_pool.shape[2]), int(block_table.shape[1])
+
+
+def la_pbd_attn_paged(cfg: Config, q, k_pool, v_pool, block_table, seq_lens, window_len: int,
+                      out, workspace: Workspace, stream=None) -> None:
+    """Window attention over paged caches: pools [num_pages, Hkv, page_size, D], block_table
+    [B, pages_per_seq] (page of each page_size run of keys)."""
+    W = int(window_len)
+    num_pages, page_size, pps = _check_paged(cfg, q, k_pool, v_pool, block_table, seq_lens, W, out)
+    _check(load().la_pbd_attn_paged(ctypes.byref(cfg), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                    _ptr(block_table), pps, page_size, num_pages, _ptr(seq_lens),
+                                    W, _ptr(out), workspace.data_ptr(), workspace.nbytes,
+                                    _stream(stream)), "la_pbd_attn_paged")
+
+
+def la_pbd_step_paged(cfg: Config, q, k_new, v_new, k_pool, v_pool, block_table, seq_lens,
+                      window_len: int, out, workspace: Workspace, stream=None) -> None:
+    """Append the window into its pages, then window attention over the paged caches (one
+    launch)."""
+    W = int(window_len)
+    num_pages, page_size, pps = _check_paged(cfg, q, k_pool, v_pool, block_table, seq_lens, W, out)
+    _check_tensor(k_new, "k_new", "bf16", (cfg.batch, W, cfg.num_kv_heads, cfg.head_dim))
+    _check_tensor(v_new, "v_new", "bf16", (cfg.batch, W, cfg.num_kv_heads, cfg.head_dim))
+    _check(load().la_pbd_step_paged(ctypes.byref(cfg), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                    _ptr(k_pool), _ptr(v_pool), _ptr(block_table), pps, page_size,
+                                    num_pages, _ptr(seq_lens), W, _ptr(out), workspace.data_ptr(),
+                                    workspace.nbytes, _stream(stream)), "la_pbd_step_paged")

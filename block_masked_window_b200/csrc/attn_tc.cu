@@ -148,6 +148,40 @@ __device__ __forceinline__ void store_pt16_impl(uint32_t prow, int c, const floa
   }
 }
 
+// Row of key j of (b, h) in the K/V tensor maps: contiguous caches, or the page pool (the key
+// must lie in one of the sequence's pages, j < pages_per_seq * page_size).
+template <bool PAGED>
+__device__ __forceinline__ int kv_row(const Problem& p, int b, int h, int j) {
+  if (!PAGED) return (b * p.Hkv + h) * p.S + j;
+  const int page = __ldg(p.block_table + (size_t)b * p.pages_per_seq + j / p.page_size);
+  return (page * p.Hkv + h) * p.page_size + (j % p.page_size);
+}
+
+// Issues the two (contiguous) or four (paged: one 64-row box per page piece) TMA loads of key
+// tile [jt, jt + 128) of segment sg into `dst`, all on barrier `fb`. Paged halves that lie
+// wholly past the segment's keys read the segment's last page instead (their rows are never
+// used), so no block-table entry beyond the sequence is touched.
+template <bool PAGED>
+__device__ __forceinline__ void load_kv_tile(const Problem& p, const Segment& sg,
+                                             const CUtensorMap* map, uint32_t dst, uint32_t fb,
+                                             int jt) {
+  if (!PAGED) {
+    const int row = (sg.b * p.Hkv + sg.h) * p.S + jt;
+    tma_load_2d(dst, map, fb, 0, row);
+    tma_load_2d(dst + kHalfBytes, map, fb, 64, row);
+    return;
+  }
+  const int jl = sg.j1 - 1;   // last key of the segment
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int j = min(jt + 64 * hr, jl);
+    const int row = kv_row<true>(p, sg.b, sg.h, j);
+    const uint32_t off = (uint32_t)hr * 64u * 128u;
+    tma_load_2d(dst + off, map, fb, 0, row);
+    tma_load_2d(dst + kHalfBytes + off, map, fb, 64, row);
+  }
+}
+
 // ---- Fused window append (step a1 inside the attention launch).
 // The window's keys [P, P + W) of a sequence (n = P + W visible keys) come from k_new / v_new.
 // The producer warp of K (or V) loads the rows that fall in key tile [jt, jt + kNT) into
@@ -167,6 +201,7 @@ __device__ __forceinline__ bool tile_window(const Problem& p, const Segment& sg,
 }
 
 // Lane l holds chunks l, l + 32, ... of the rows [w0, w1) (16 chunks of 16 bytes per row).
+template <bool PAGED>
 __device__ __forceinline__ void window_load_append(const Problem& p, const Segment& sg,
                                                    const __nv_bfloat16* src,
                                                    __nv_bfloat16* cache, int w0, int w1,
@@ -182,7 +217,7 @@ __device__ __forceinline__ void window_load_append(const Problem& p, const Segme
           src + (((size_t)sg.b * p.W + w) * p.Hkv + sg.h) * kHeadDim) + ch;
       v[u] = __ldg(s);
       uint4* d = reinterpret_cast<uint4*>(
-          cache + (((size_t)sg.b * p.Hkv + sg.h) * p.S + (size_t)(P + w)) * kHeadDim) + ch;
+          cache + (size_t)kv_row<PAGED>(p, sg.b, sg.h, P + w) * kHeadDim) + ch;
       *d = v[u];
     }
   }
@@ -209,7 +244,7 @@ __device__ __forceinline__ void window_patch(uint32_t tile, const Problem& p, co
 
 }  // namespace
 
-template <int NQ, bool CAUSAL>
+template <int NQ, bool CAUSAL, bool PAGED>
 __global__ void __launch_bounds__(kThreadsTc, 1)
     pbd_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                        const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
@@ -318,10 +353,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
       const int nt = tiles_of(sg);
       for (int t = 0; t < nt; ++t, ++g) {
-        const int row = row0 + t * kNT, jt = sg.j0 + t * kNT;
+        const int jt = sg.j0 + t * kNT;
         const int ks = g % kKStages, ku = g / kKStages;
         int w0 = 0, w1 = 0;
         const bool fuse = p.k_new != nullptr && tile_window(p, sg, jt, w0, w1);
@@ -332,8 +366,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t dk = sK + ks * kTileBytes;
             const uint32_t fb = bar((fuse ? kBarKRaw : kBarKFull) + ks);
             mbar_expect_tx(fb, (uint32_t)kTileBytes);
-            tma_load_2d(dk, &tmk, fb, 0, row);
-            tma_load_2d(dk + kHalfBytes, &tmk, fb, 64, row);
+            load_kv_tile<PAGED>(p, sg, &tmk, dk, fb, jt);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -341,7 +374,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (fuse) {
           // While the tile is in flight: fetch the window rows and append them to the cache.
           uint4 win[kWinRegs];
-          window_load_append(p, sg, p.k_new, p.kc, w0, w1, lane, win);
+          window_load_append<PAGED>(p, sg, p.k_new, p.kc, w0, w1, lane, win);
           const uint32_t fb = bar(kBarKRaw + ks);
           if (lane == 0 && !mbar_wait(fb, (raw_par >> ks) & 1u, ctl)) {
             mbar_drain(fb, (raw_par >> ks) & 1u, 100000000LL);
@@ -374,10 +407,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     uint32_t raw_par = 0;
     bool ok = true;
     while (ok && it.next(p, pre, blockIdx.x, sg)) {
-      const int row0 = (sg.b * p.Hkv + sg.h) * p.S + sg.j0;
       const int nt = tiles_of(sg);
       for (int t = 0; t < nt; ++t, ++g) {
-        const int row = row0 + t * kNT, jt = sg.j0 + t * kNT;
+        const int jt = sg.j0 + t * kNT;
         const int vs = g % vstages, vu = g / vstages;
         int w0 = 0, w1 = 0;
         const bool fuse = p.v_new != nullptr && tile_window(p, sg, jt, w0, w1);
@@ -388,8 +420,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const uint32_t dv = sV + vs * kTileBytes;
             const uint32_t fb = bar((fuse ? kBarVRaw : kBarVFull) + vs);
             mbar_expect_tx(fb, (uint32_t)kTileBytes);
-            tma_load_2d(dv, &tmv, fb, 0, row);
-            tma_load_2d(dv + kHalfBytes, &tmv, fb, 64, row);
+            load_kv_tile<PAGED>(p, sg, &tmv, dv, fb, jt);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -397,7 +428,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (fuse) {
           // While the tile is in flight: fetch the window rows and append them to the cache.
           uint4 win[kWinRegs];
-          window_load_append(p, sg, p.v_new, p.vc, w0, w1, lane, win);
+          window_load_append<PAGED>(p, sg, p.v_new, p.vc, w0, w1, lane, win);
           const uint32_t fb = bar(kBarVRaw + vs);
           if (lane == 0 && !mbar_wait(fb, (raw_par >> vs) & 1u, ctl)) {
             mbar_drain(fb, (raw_par >> vs) & 1u, 100000000LL);
@@ -858,7 +889,8 @@ int tc_tile_keys() { return kNT; }
 static int tc_nq(int R) { return round_up(R, 16); }
 
 // V ring depth and Q buffers that fit: the V ring depth matters most (a V tile is held until
-// its PV product completes), a second Q buffer only hides segment changes.
+// its PV product completes), a second Q buffer only hides segment changes (measured: no gain
+// on a ragged batch of 64 sequences when it costs a V stage).
 static int tc_ring(int nq, int B) {
   const int limit = 227 * 1024 - 1024;
   const int options[5][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}, {1, 1}};
@@ -873,16 +905,16 @@ size_t tc_smem_bytes(int R, int B) {
   return ring ? (size_t)1024 + tc_layout(nq, ring & 0xff, ring >> 8, B).end : 0;
 }
 
-template <int NQ, bool CAUSAL>
+template <int NQ, bool CAUSAL, bool PAGED>
 static cudaError_t launch_nq(const Problem& p, const CUtensorMap& k, const CUtensorMap& v,
                              const CUtensorMap& q, const CUtensorMap& o, cudaStream_t stream) {
   const int ring = tc_ring(NQ, p.B);
   if (ring == 0) return cudaErrorInvalidValue;
   const size_t smem = (size_t)1024 + tc_layout(NQ, ring & 0xff, ring >> 8, p.B).end;
-  cudaError_t e = cudaFuncSetAttribute(pbd_attn_tc_kernel<NQ, CAUSAL>,
+  cudaError_t e = cudaFuncSetAttribute(pbd_attn_tc_kernel<NQ, CAUSAL, PAGED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(pbd_attn_tc_kernel<NQ, CAUSAL>, dim3(p.num_ctas), dim3(kThreadsTc), smem,
+  return launch_pdl(pbd_attn_tc_kernel<NQ, CAUSAL, PAGED>, dim3(p.num_ctas), dim3(kThreadsTc), smem,
                     stream, k, v, q, o, p, ring);
 }
 
@@ -893,13 +925,23 @@ cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tma
   const CUtensorMap& q = *static_cast<const CUtensorMap*>(tmap_q);
   const CUtensorMap& o = *static_cast<const CUtensorMap*>(tmap_o);
   const bool causal = row_limits(p);   // per-row key limits
+  // Paged caches get their own instantiations so that the contiguous kernels' code (and its
+  // instruction-cache footprint on the latency-bound single-tile path) is unchanged.
+  const bool paged = p.block_table != nullptr;
+#define LA_TC_CASE(N)                                                                      \
+  case N:                                                                                  \
+    if (paged) return causal ? launch_nq<N, true, true>(p, k, v, q, o, stream)            \
+                             : launch_nq<N, false, true>(p, k, v, q, o, stream);          \
+    return causal ? launch_nq<N, true, false>(p, k, v, q, o, stream)                      \
+                  : launch_nq<N, false, false>(p, k, v, q, o, stream);
   switch (tc_nq(p.R)) {
-    case 16: return causal ? launch_nq<16, true>(p, k, v, q, o, stream) : launch_nq<16, false>(p, k, v, q, o, stream);
-    case 32: return causal ? launch_nq<32, true>(p, k, v, q, o, stream) : launch_nq<32, false>(p, k, v, q, o, stream);
-    case 48: return causal ? launch_nq<48, true>(p, k, v, q, o, stream) : launch_nq<48, false>(p, k, v, q, o, stream);
-    case 64: return causal ? launch_nq<64, true>(p, k, v, q, o, stream) : launch_nq<64, false>(p, k, v, q, o, stream);
+    LA_TC_CASE(16)
+    LA_TC_CASE(32)
+    LA_TC_CASE(48)
+    LA_TC_CASE(64)
     default: return cudaErrorInvalidValue;
   }
+#undef LA_TC_CASE
 }
 
 }  // namespace la

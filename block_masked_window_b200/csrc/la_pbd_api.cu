@@ -165,13 +165,26 @@ namespace {
 // Attention launch (attention kernel + merge) for validated arguments. With k_new / v_new
 // non-null the caller has chosen the tcgen05 kernel, which then also appends the window
 // (caches written through k_cache / v_cache).
+// Paged caches for attn_launch (null block_table: contiguous caches).
+struct Paging {
+  const int32_t* block_table = nullptr;
+  int pages_per_seq = 0, page_size = 0, num_pages = 0;
+};
+
 la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* seq_lens,
                       const int32_t* window_lens, int32_t W, void* out, void* workspace,
-                      const void* k_new, const void* v_new, void* stream) {
+                      const void* k_new, const void* v_new, void* stream,
+                      const Paging& pg = Paging()) {
   Problem p;
   fill_problem(cfg, W, &p);
   p.window_lens = window_lens;
+  if (pg.block_table) {
+    p.block_table = pg.block_table;
+    p.pages_per_seq = pg.pages_per_seq;
+    p.page_size = pg.page_size;
+    p.S = pg.pages_per_seq * pg.page_size;   // key capacity of a sequence
+  }
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k_cache);
   p.v = static_cast<const __nv_bfloat16*>(v_cache);
@@ -188,13 +201,16 @@ la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
   cudaError_t e = cudaSuccess;
   const int algo = pick_algo(cfg, p.R);
   if (k_new && algo != LA_ALGO_TCGEN05) return LA_ERR_INVALID_ARG;
+  if (pg.block_table && algo != LA_ALGO_TCGEN05) return LA_ERR_UNSUPPORTED;
   if (algo == LA_ALGO_TCGEN05) {
     p.k_new = static_cast<const __nv_bfloat16*>(k_new);
     p.v_new = static_cast<const __nv_bfloat16*>(v_new);
     p.kc = const_cast<__nv_bfloat16*>(p.k);
     p.vc = const_cast<__nv_bfloat16*>(p.v);
     la::TmaMaps maps;
-    if (la::make_tma_maps(p, &maps) != cudaSuccess) return LA_ERR_CUDA;
+    const long long pool_rows =
+        pg.block_table ? (long long)pg.num_pages * p.Hkv * pg.page_size : 0;
+    if (la::make_tma_maps(p, &maps, pool_rows) != cudaSuccess) return LA_ERR_CUDA;
     p.unit = la::tc_tile_keys();
     p.c_min = 1;
     p.num_ctas = grid_for(p, sms * la::tc_ctas_per_sm());
@@ -349,6 +365,59 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
   if (la::make_prefill_maps(p, &mq, &mk, &mv) != cudaSuccess) return LA_ERR_CUDA;
   cudaError_t e = la::launch_prefill_tc(p, &mq, &mk, &mv, (cudaStream_t)stream);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+static la_status check_paging(const la_pbd_cfg* cfg, int32_t W, const int32_t* block_table,
+                              int32_t pages_per_seq, int32_t page_size, int32_t num_pages) {
+  if (!block_table || !aligned(block_table, 4)) return LA_ERR_INVALID_ARG;
+  if (pages_per_seq < 1 || num_pages < 1 || page_size < 64 || page_size % 64 != 0)
+    return LA_ERR_INVALID_ARG;
+  if ((long long)num_pages * cfg->num_kv_heads * page_size >= (1LL << 31)) return LA_ERR_UNSUPPORTED;
+  if ((long long)cfg->batch * cfg->num_kv_heads * pages_per_seq * page_size >= (1LL << 31))
+    return LA_ERR_UNSUPPORTED;
+  if (pick_algo(cfg, W * (cfg->num_q_heads / cfg->num_kv_heads)) != LA_ALGO_TCGEN05)
+    return LA_ERR_UNSUPPORTED;
+  return LA_OK;
+}
+
+la_status la_pbd_attn_paged(const la_pbd_cfg* cfg, const void* q, const void* k_pool,
+                            const void* v_pool, const int32_t* block_table,
+                            int32_t pages_per_seq, int32_t page_size, int32_t num_pages,
+                            const int32_t* seq_lens, int32_t W, void* out, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  la_status st = check_attn_args(cfg, q, k_pool, v_pool, seq_lens, W, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  st = check_paging(cfg, W, block_table, pages_per_seq, page_size, num_pages);
+  if (st != LA_OK) return st;
+  Paging pg;
+  pg.block_table = block_table;
+  pg.pages_per_seq = pages_per_seq;
+  pg.page_size = page_size;
+  pg.num_pages = num_pages;
+  return attn_launch(cfg, q, k_pool, v_pool, seq_lens, nullptr, W, out, workspace, nullptr,
+                     nullptr, stream, pg);
+}
+
+la_status la_pbd_step_paged(const la_pbd_cfg* cfg, const void* q, const void* k_new,
+                            const void* v_new, void* k_pool, void* v_pool,
+                            const int32_t* block_table, int32_t pages_per_seq,
+                            int32_t page_size, int32_t num_pages, const int32_t* seq_lens,
+                            int32_t W, void* out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  la_status st = check_attn_args(cfg, q, k_pool, v_pool, seq_lens, W, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  st = check_paging(cfg, W, block_table, pages_per_seq, page_size, num_pages);
+  if (st != LA_OK) return st;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return LA_ERR_INVALID_ARG;
+  Paging pg;
+  pg.block_table = block_table;
+  pg.pages_per_seq = pages_per_seq;
+  pg.page_size = page_size;
+  pg.num_pages = num_pages;
+  return attn_launch(cfg, q, k_pool, v_pool, seq_lens, nullptr, W, out, workspace, k_new,
+                     v_new, stream, pg);
 }
 
 la_status la_pbd_check(void* workspace, void* stream) {

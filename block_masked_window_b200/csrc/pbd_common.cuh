@@ -39,6 +39,11 @@ struct Problem {
   const __nv_bfloat16* v;       // [B, Hkv, S, D]
   const int32_t* seq_lens;      // [B]
   const int32_t* window_lens;   // [B] window length W_b <= W of each sequence, or null (all W)
+  // Paged caches (tcgen05 kernel only): k and v are page pools [num_pages, Hkv, page_size, D]
+  // and key j of sequence b lives in page block_table[b * pages_per_seq + j / page_size];
+  // null block_table = contiguous caches [B, Hkv, S, D].
+  const int32_t* block_table;
+  int pages_per_seq, page_size;
   __nv_bfloat16* out;           // [B, W, Hq, D]
   // Fused window append (tcgen05 kernel only; null otherwise): the window's keys/values are
   // read from k_new / v_new [B, W, Hkv, D] and written into the caches kc / vc (= k, v).

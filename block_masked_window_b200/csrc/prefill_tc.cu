@@ -62,6 +62,13 @@ constexpr int kOffMisc = kOffBar + kBNum * 8;
 constexpr int kPfSmem = kOffMisc + 16;
 constexpr size_t kPfSmemAlloc = (size_t)kPfSmem + 1024;   // + alignment slack
 
+// 8 bf16 probabilities (keys 8 k8 .. 8 k8 + 7) of row r into the swizzled K-major P tile.
+__device__ __forceinline__ void store_p16(uint32_t prow, int k8, int r, const uint32_t (&pk)[4]) {
+  const uint32_t a = prow + (uint32_t)((k8 >> 3) * kPHalf + (((k8 & 7) ^ (r & 7)) << 4));
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[0]), "r"(pk[1]),
+               "r"(pk[2]), "r"(pk[3]));
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kPfThreads, 1)
@@ -257,18 +264,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int c = 0; c < kBN / 32; ++c) tmem_ld32(s_addr + 32 * c, x + 32 * c);
       tc_wait_ld();
       // Tiles wholly below this row's limit need no mask (all but the last one or two).
+      // (Eight independent partial maxima: one softmax warp per scheduler, so a single
+      // 128-long dependency chain would leave the issue slots idle.)
       const bool full = j0 + kBN <= lim;
-      float mt = -INFINITY;
-      if (full) {
+      if (!full) {
 #pragma unroll
-        for (int e = 0; e < kBN; ++e) mt = fmaxf(mt, x[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < kBN; ++e) {
+        for (int e = 0; e < kBN; ++e)
           if (j0 + e >= lim) x[e] = -INFINITY;
-          mt = fmaxf(mt, x[e]);
-        }
       }
+      float mp[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mp[u] = x[u];
+#pragma unroll
+      for (int e = 8; e < kBN; ++e) mp[e & 7] = fmaxf(mp[e & 7], x[e]);
+      float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       mt *= c2;   // log2 units (c2 > 0)
       // Lazy reference: raise it only when a score exceeds it by more than 2^8.
       const bool raise = mt > m_ref + kPfLazy || (m_ref == -INFINITY && mt > -INFINITY);
@@ -299,10 +309,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + (t & 1)), ((t - 2) >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
       }
-      // p = 2^(x c2 - m_ref) (masked scores are -inf: p = 0), bf16 into the swizzled
-      // K-major P tile, 8 keys per 16-byte store.
+      // p = 2^(x c2 - m_ref), bf16 into the swizzled K-major P tile, 8 keys per 16-byte
+      // store.
       const uint32_t prow = sP + (t & 1) * kPTile + (uint32_t)r * 128u;
       const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // (Masked scores are -inf: ex2.approx gives exactly 0 for them.)
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums (see the maxima)
 #pragma unroll
       for (int k8 = 0; k8 < kBN / 8; ++k8) {
         uint32_t pk[4];
@@ -310,14 +322,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int e = 0; e < 8; e += 2) {
           const float a = fast_exp2(fmaf(x[8 * k8 + e], c2, -mref));
           const float bq = fast_exp2(fmaf(x[8 * k8 + e + 1], c2, -mref));
-          l += a + bq;
+          ls[e >> 1] += a + bq;
           __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bq);
           pk[e >> 1] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        const uint32_t a = prow + (uint32_t)((k8 >> 3) * kPHalf + (((k8 & 7) ^ (r & 7)) << 4));
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[0]), "r"(pk[1]),
-                     "r"(pk[2]), "r"(pk[3]));
+        store_p16(prow, k8, r, pk);
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       // Keys past the visible range in the last tile: zero their V rows so that 0 * x
       // cannot become NaN in the product (those rows may hold anything).
       const int valid = min(kBN, kmax - j0);

@@ -43,14 +43,16 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-inline cudaError_t make_tma_maps(const Problem& p, TmaMaps* m) {
+// pool_rows > 0: paged caches, K/V are page pools of pool_rows rows read as 64-row boxes (one
+// box per page piece of a key tile).
+inline cudaError_t make_tma_maps(const Problem& p, TmaMaps* m, long long pool_rows = 0) {
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  const cuuint64_t rows = (cuuint64_t)p.B * p.Hkv * p.S;
+  const cuuint64_t rows = pool_rows > 0 ? (cuuint64_t)pool_rows : (cuuint64_t)p.B * p.Hkv * p.S;
   {
     cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, rows};
     cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kTileKeys};
+    cuuint32_t box[2] = {64, (cuuint32_t)(pool_rows > 0 ? 64 : kTileKeys)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&m->k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)p.k, dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

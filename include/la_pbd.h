@@ -188,6 +188,30 @@ la_status la_pbd_step_varwin(const la_pbd_cfg* cfg, const void* q, const void* k
                              size_t workspace_bytes, void* stream);
 
 /*
+ * Paged KV cache (tcgen05 kernel only, i.e. W * Hq/Hkv <= 64 and algo != LA_ALGO_SIMT, else
+ * LA_ERR_UNSUPPORTED). The caches are page pools
+ *   k_pool, v_pool  bf16 [num_pages, Hkv, page_size, D]
+ *   block_table     device int32 [B, pages_per_seq]: key j of sequence b lives in page
+ *                   block_table[b][j / page_size], row j % page_size
+ * page_size a multiple of 64 (each 128-key tile is read as 64-row boxes). A sequence holds
+ * at most pages_per_seq * page_size keys (this replaces cfg->max_seq for the capacity check);
+ * the table entries of pages [0, ceil((P_b + W) / page_size)) must be valid pages, later
+ * entries are never read. Otherwise as la_pbd_attn / la_pbd_step (the step appends the window
+ * rows into their pages, fused into the attention launch).
+ */
+la_status la_pbd_attn_paged(const la_pbd_cfg* cfg, const void* q, const void* k_pool,
+                            const void* v_pool, const int32_t* block_table,
+                            int32_t pages_per_seq, int32_t page_size, int32_t num_pages,
+                            const int32_t* seq_lens, int32_t window_len, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+la_status la_pbd_step_paged(const la_pbd_cfg* cfg, const void* q, const void* k_new,
+                            const void* v_new, void* k_pool, void* v_pool,
+                            const int32_t* block_table, int32_t pages_per_seq,
+                            int32_t page_size, int32_t num_pages, const int32_t* seq_lens,
+                            int32_t window_len, void* out, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
  * Block-causal prefill attention (the block mask of block-diffusion decoding over whole
  * sequences; the PBD window is the last block of it): token i of sequence b attends key j
  * when j <= i or when both lie in the same block of block_size consecutive tokens, i.e. j <
