@@ -9,17 +9,20 @@
 // see, flash-attention style, on the tensor cores:
 //   S = Q K^T  (M = 128 query rows, N = 128 keys,     K = 128 channels) -> TMEM fp32, 2 bufs
 //   O += P V   (M = 128 query rows, N = 128 channels, K = 128 keys)     -> TMEM fp32
-// Thread r of the 128 softmax threads owns query row r (TMEM lane r): it reads its scores
-// from TMEM, keeps its running reference maximum and row sum in registers, writes its row of
-// P (bf16) into shared memory in the 128-byte-swizzled K-major layout the MMA reads, and at
-// the end normalises its O row and stores it. The reference maximum is lazy (raised only
-// when a score exceeds it by 2^8); a warp whose lanes raise it rescales their O rows in TMEM
-// after the previous PV product has completed.
+// Two softmax threads own query row r (TMEM lane r), one per 64-column half of the key tile
+// (and of O): each reads its 64 scores from TMEM, the pair exchanges its half maxima (and at
+// the end its half sums) through shared memory, both keep the same running reference maximum
+// in registers, and each writes its half of the row of P (bf16) into shared memory in the
+// 128-byte-swizzled K-major layout the MMA reads and normalises and stores its half of the O
+// row. The reference maximum is lazy (raised only when a score exceeds it by 2^8); a warp
+// whose lanes raise it rescales their O columns in TMEM after the previous PV product has
+// completed.
 //
-// Roles (224 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 6 TMA for the V
-// ring, warp 1 TMEM owner and MMA issuer, warps 2..5 softmax. Query tiles are scheduled
-// longest first (the last tiles see the most keys). Every wait is bounded (sticky timeout
-// flag, drain, TMEM freed, return).
+// Roles (352 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 10 TMA for the V
+// ring, warp 1 TMEM owner and MMA issuer, warps 2..9 softmax (warps w and w + 4 share the TMEM
+// lane quarter w % 4: two warps per scheduler hide each other's latencies). Query tiles are
+// scheduled longest first (the last tiles see the most keys). Every wait is bounded (sticky
+// timeout flag, drain, TMEM freed, return).
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 #include "tc_util.cuh"
@@ -32,7 +35,7 @@ using namespace tc;
 
 constexpr int kBM = 128;                 // query rows per CTA
 constexpr int kBN = 128;                 // keys per tile
-constexpr int kPfThreads = 224;
+constexpr int kPfThreads = 352;         // 11 warps
 constexpr int kPfStages = 2;             // K and V ring depth
 constexpr int kPHalf = 128 * 128;        // one 64-column half of a 128-row bf16 tile (16 KB)
 constexpr int kPTile = 2 * kPHalf;       // 32 KB
@@ -59,8 +62,12 @@ constexpr int kOffV = kOffK + kPfStages * kPTile;
 constexpr int kOffP = kOffV + kPfStages * kPTile;
 constexpr int kOffBar = kOffP + 2 * kPTile;
 constexpr int kOffMisc = kOffBar + kBNum * 8;
-constexpr int kPfSmem = kOffMisc + 16;
+constexpr int kOffX = kOffMisc + 16;              // [2 halves][128 rows] floats: row maxima / sums
+constexpr int kPfSmem = kOffX + 2 * 128 * 4;
 constexpr size_t kPfSmemAlloc = (size_t)kPfSmem + 1024;   // + alignment slack
+
+// Named barrier 1 over the 256 softmax threads.
+__device__ __forceinline__ void pf_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // 8 bf16 probabilities (keys 8 k8 .. 8 k8 + 7) of row r into the swizzled K-major P tile.
 __device__ __forceinline__ void store_p16(uint32_t prow, int k8, int r, const uint32_t (&pk)[4]) {
@@ -104,7 +111,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBSFull + s), 1);
-      mbar_init(bar(kBPFull + s), 128);
+      mbar_init(bar(kBPFull + s), 256);
       mbar_init(bar(kBOFull + s), 1);
     }
     mbar_init(bar(kBDrain), 1);
@@ -156,7 +163,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       mbar_drain(bar(kBQFull), 0, 100000000LL);
     }
-  } else if (nk > 0 && warp == 6) {
+  } else if (nk > 0 && warp == 10) {
     // ------------------------------------------------------------------ TMA: V
     if (lane == 0) {
       bool ok = true;
@@ -242,44 +249,51 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       umma_commit(bar(kBDrain));
       mbar_drain(bar(kBDrain), 0, 100000000LL);
     }
-  } else if (warp >= 2 && warp <= 5) {
+  } else if (warp >= 2 && warp <= 9) {
     // ------------------------------------------------------------------ softmax warps
     const int sub = warp & 3;
+    const int half = (warp - 2) >> 2;              // 64-column half of the tile (and of O)
     const int r = 32 * sub + lane;                 // query row of this thread (TMEM lane)
     const int i = i0 + r;
+    const int st = 128 * half + r;                 // softmax thread index 0..255
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * sub) << 16);
     const int lim = (i < Tb) ? min(Tb, (i / p.bs + 1) * p.bs) : 0;   // keys [0, lim)
     const float c2 = p.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;
+    float* xs = reinterpret_cast<float*>(base + kOffX);   // [2][128] half maxima, then sums
+    float m_ref = -INFINITY, l = 0.f;                       // l: this half's sum
     bool ok = true;
     for (int t = 0; t < nk; ++t) {
-      const int j0 = t * kBN;
-      const uint32_t s_addr = lane_addr + kColS + (uint32_t)((t & 1) * kBN);
+      const int j0 = t * kBN + 64 * half;          // first key of this thread's half
+      const uint32_t s_addr = lane_addr + kColS + (uint32_t)((t & 1) * kBN + 64 * half);
       // (Every lane waits on the same barrier; the vote keeps the error path warp-uniform.)
       if (!__all_sync(0xffffffffu, mbar_wait(bar(kBSFull + (t & 1)), (t >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
-      // The row's 128 scores, one TMEM read (4 x 32 columns, one wait).
-      float x[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(s_addr + 32 * c, x + 32 * c);
+      // This half's 64 scores: two 32-column TMEM reads, one wait.
+      float x[64];
+      tmem_ld32(s_addr, x);
+      tmem_ld32(s_addr + 32, x + 32);
       tc_wait_ld();
-      // Tiles wholly below this row's limit need no mask (all but the last one or two).
-      // (Eight independent partial maxima: one softmax warp per scheduler, so a single
-      // 128-long dependency chain would leave the issue slots idle.)
-      const bool full = j0 + kBN <= lim;
+      // Halves wholly below this row's limit need no mask (all but the last one or two).
+      // (Eight independent partial maxima: a single 64-long dependency chain would leave the
+      // issue slots idle.)
+      const bool full = j0 + 64 <= lim;
       if (!full) {
 #pragma unroll
-        for (int e = 0; e < kBN; ++e)
+        for (int e = 0; e < 64; ++e)
           if (j0 + e >= lim) x[e] = -INFINITY;
       }
       float mp[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mp[u] = x[u];
 #pragma unroll
-      for (int e = 8; e < kBN; ++e) mp[e & 7] = fmaxf(mp[e & 7], x[e]);
-      float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      mt *= c2;   // log2 units (c2 > 0)
+      for (int e = 8; e < 64; ++e) mp[e & 7] = fmaxf(mp[e & 7], x[e]);
+      const float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      // The row's maximum from both halves (both threads of the row then take the same
+      // decisions below).
+      xs[st] = mh;
+      pf_bar();
+      float mt = fmaxf(mh, xs[st ^ 128]) * c2;    // log2 units (c2 > 0)
       // Lazy reference: raise it only when a score exceeds it by more than 2^8.
       const bool raise = mt > m_ref + kPfLazy || (m_ref == -INFINITY && mt > -INFINITY);
       float alpha = 1.f;
@@ -288,19 +302,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         l *= alpha;
         m_ref = mt;
       }
-      // Rows whose reference moved rescale their O row (warp-uniform TMEM access), once
-      // the previous PV product is complete.
+      // Rows whose reference moved rescale their half of the O row (warp-uniform TMEM
+      // access), once the previous PV product is complete.
       if (t > 0 && __any_sync(0xffffffffu, raise)) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 128 / 16; ++c) {
+        for (int c = 0; c < 64 / 16; ++c) {
           float o[16];
-          tmem_ld16(lane_addr + kColO + 16 * c, o);
+          const uint32_t col = kColO + 64 * half + 16 * c;
+          tmem_ld16(lane_addr + col, o);
           tc_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] *= alpha;
-          tmem_st16(lane_addr + kColO + 16 * c, o);
+          tmem_st16(lane_addr + col, o);
         }
         tc_wait_st();
       }
@@ -309,14 +324,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + (t & 1)), ((t - 2) >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
       }
-      // p = 2^(x c2 - m_ref), bf16 into the swizzled K-major P tile, 8 keys per 16-byte
-      // store.
+      // p = 2^(x c2 - m_ref), bf16 into this half of the swizzled K-major P row, 8 keys per
+      // 16-byte store. (Masked scores are -inf: ex2.approx gives exactly 0 for them.)
       const uint32_t prow = sP + (t & 1) * kPTile + (uint32_t)r * 128u;
       const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // (Masked scores are -inf: ex2.approx gives exactly 0 for them.)
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums (see the maxima)
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k8 = 0; k8 < kBN / 8; ++k8) {
+      for (int k8 = 0; k8 < 8; ++k8) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
@@ -326,37 +340,43 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bq);
           pk[e >> 1] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        store_p16(prow, k8, r, pk);
+        store_p16(prow, 8 * half + k8, r, pk);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       // Keys past the visible range in the last tile: zero their V rows so that 0 * x
       // cannot become NaN in the product (those rows may hold anything).
-      const int valid = min(kBN, kmax - j0);
+      const int valid = min(kBN, kmax - t * kBN);
       if (valid < kBN) {
         const int s = t % kPfStages;
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kBVFull + s), (t / kPfStages) & 1, ctl))) { ok = false; break; }
         const uint32_t vbase = sV + s * kPTile;
-        for (int idx = r; idx < (kBN - valid) * 16; idx += 128) {
+        for (int idx = st; idx < (kBN - valid) * 16; idx += 256) {
           const int rr = valid + (idx >> 4), ch = idx & 15;
           const uint32_t a = vbase + (ch >> 3) * kPHalf + rr * 128 + (ch & 7) * 16;
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(0u), "r"(0u),
                        "r"(0u), "r"(0u));
         }
       }
+      // Both halves have read the exchanged maxima before the next tile overwrites them.
+      pf_bar();
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(bar(kBPFull + (t & 1)));
     }
-    // Epilogue: O row / l as bf16, straight to global memory (256 contiguous bytes per row).
+    // Epilogue: the row sum from both halves; each thread stores its 64 channels (128 bytes)
+    // of O / l as bf16.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBOFull + ((nk - 1) & 1)), ((nk - 1) >> 1) & 1, ctl));
     tc_fence_after();
-    __nv_bfloat16* dst = p.out + (((size_t)b * p.T + i) * p.Hq + h) * kHeadDim;
-    const float inv = (ok && i < Tb && l > 0.f) ? 1.f / l : 0.f;
+    xs[st] = l;
+    pf_bar();
+    const float lrow = l + xs[st ^ 128];
+    __nv_bfloat16* dst = p.out + (((size_t)b * p.T + i) * p.Hq + h) * kHeadDim + 64 * half;
+    const float inv = (ok && i < Tb && lrow > 0.f) ? 1.f / lrow : 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 128 / 16; ++c) {
+    for (int c = 0; c < 64 / 16; ++c) {
       float o[16];
       if (ok) {   // (warp-uniform)
-        tmem_ld16(lane_addr + kColO + 16 * c, o);
+        tmem_ld16(lane_addr + kColO + 64 * half + 16 * c, o);
         tc_wait_ld();
       } else {
 #pragma unroll
@@ -375,13 +395,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     }
   }
-  if (nk == 0 && warp >= 2 && warp <= 5) {
-    // No valid row in this tile: the owned rows of `out` are zeros.
-    const int r = 32 * (warp & 3) + lane;
+  if (nk == 0 && warp >= 2 && warp <= 9) {
+    // No valid row in this tile: the owned rows of `out` are zeros (each thread 64 channels).
+    const int r = 32 * (warp & 3) + lane, half = (warp - 2) >> 2;
     if (r < rows_here) {
-      uint4* d4 = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.T + i0 + r) * p.Hq + h) * kHeadDim);
+      uint4* d4 = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.T + i0 + r) * p.Hq + h) * kHeadDim +
+                                           64 * half);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) d4[c] = make_uint4(0u, 0u, 0u, 0u);
+      for (int c = 0; c < 8; ++c) d4[c] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   tc_fence_before();
