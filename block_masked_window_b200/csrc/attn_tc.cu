@@ -315,8 +315,52 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // Everything above is on-chip; from here on global memory written by the previous kernel
-  // of the stream is read.
+  // Before the wait (small batches, contiguous caches): guess this CTA's first key tiles from
+  // the current seq_lens and have them and Q fetched into L2 while the previous kernel
+  // finishes. The guess is only a hint: the reads bypass L1 (so no stale line can be hit
+  // after the wait), a wrong guess only wastes the prefetch, and the plan is made again from
+  // the values read after the wait.
+  if (!PAGED && warp == 0 && p.B <= 32) {
+    int u = 0;
+    if (lane < p.B) {
+      const int P = __ldcg(p.seq_lens + lane);
+      const int w = p.window_lens ? __ldcg(p.window_lens + lane) : p.W;
+      const bool valid = P >= 0 && w >= 1 && w <= p.W && (long long)P + w <= (long long)p.S;
+      u = valid ? units_of(p, P + w) : 0;
+    }
+    int incl = u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int excl = incl - u;
+    const long long Tg = (long long)p.Hkv * __shfl_sync(0xffffffffu, incl, 31);
+    const long long Cg = Tg > 0 ? plan_chunk(p, Tg) : 1;
+    const long long pos = (long long)blockIdx.x * Cg;
+    const unsigned starts = __ballot_sync(0xffffffffu, lane < p.B && u > 0 &&
+                                                           (long long)p.Hkv * excl <= pos);
+    const int bb = starts ? 31 - __clz(starts) : 0;
+    const int ub = __shfl_sync(0xffffffffu, u, bb), pb = __shfl_sync(0xffffffffu, excl, bb);
+    if (lane == 0 && pos < Tg && starts != 0u && ub > 0) {
+      const long long off = pos - (long long)p.Hkv * pb;
+      const int hh = (int)(off / ub), t0 = (int)(off - (long long)hh * ub);
+      if (hh < p.Hkv) {
+        tma_prefetch_3d(&tmq, 0, hh * p.G, bb * p.W);
+        tma_prefetch_3d(&tmq, 64, hh * p.G, bb * p.W);
+        const int nt = (int)min((long long)(ub - t0), min(Cg, 2LL));
+        for (int t = 0; t < nt; ++t) {
+          const int row = (bb * p.Hkv + hh) * p.S + (t0 + t) * kNT;
+          tma_prefetch_2d(&tmk, 0, row);
+          tma_prefetch_2d(&tmk, 64, row);
+          tma_prefetch_2d(&tmv, 0, row);
+          tma_prefetch_2d(&tmv, 64, row);
+        }
+      }
+    }
+  }
+  // Everything above is on-chip (or an L2 hint); from here on global memory written by the
+  // previous kernel of the stream is read.
   pdl_wait();
   plan_prefix(p, pre, warp_tot);
   fence_async_smem();

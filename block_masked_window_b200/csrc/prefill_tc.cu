@@ -9,14 +9,18 @@
 // see, flash-attention style, on the tensor cores:
 //   S = Q K^T  (M = 128 query rows, N = 128 keys,     K = 128 channels) -> TMEM fp32, 2 bufs
 //   O += P V   (M = 128 query rows, N = 128 channels, K = 128 keys)     -> TMEM fp32
-// Two softmax threads own query row r (TMEM lane r), one per 64-column half of the key tile
-// (and of O): each reads its 64 scores from TMEM, the pair exchanges its half maxima (and at
-// the end its half sums) through shared memory, both keep the same running reference maximum
-// in registers, and each writes its half of the row of P (bf16) into shared memory in the
-// 128-byte-swizzled K-major layout the MMA reads and normalises and stores its half of the O
-// row. The reference maximum is lazy (raised only when a score exceeds it by 2^8); a warp
-// whose lanes raise it rescales their O columns in TMEM after the previous PV product has
-// completed.
+// The 128 keys of each tile are split into two halves that are processed independently, as
+// two interleaved split-KV streams: half h's probabilities multiply V rows [64h, 64h + 64)
+// into their own accumulator O_h (TMEM: two S buffers and O_0, O_1 fill the 512 columns),
+// with their own reference maximum and row sum, and the two are merged once at the end. Two
+// softmax threads own query row r (TMEM lane r), one per key half: each reads its 64 scores
+// from TMEM, keeps its lazy reference maximum (raised only when a score exceeds it by 2^8;
+// the warp then rescales its O_h rows after the previous PV product has completed) and row
+// sum in registers, and writes its half of the row of P (bf16) into shared memory in the
+// 128-byte-swizzled K-major layout the MMA reads. With no exchange between the halves per
+// tile, the two warps sharing a scheduler drift apart, so one's exponentials overlap the
+// other's maxima and TMEM reads. At the end the pair merges (m, l, O_0, O_1) and each thread
+// normalises and stores 64 of the row's 128 output channels.
 //
 // Roles (352 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 10 TMA for the V
 // ring, warp 1 TMEM owner and MMA issuer, warps 2..9 softmax (warps w and w + 4 share the TMEM
@@ -42,7 +46,7 @@ constexpr int kPTile = 2 * kPHalf;       // 32 KB
 constexpr float kPfLazy = 8.f;           // log2 units
 constexpr int kPfTmemCols = 512;
 constexpr int kColS = 0;                 // S: 2 buffers x 128 columns
-constexpr int kColO = 2 * kBN;           // O: 128 columns
+constexpr int kColO = 2 * kBN;           // O of key half 0 (128 columns), then of key half 1
 
 constexpr int kBQFull = 0;
 constexpr int kBKFull = 1;                        // [kPfStages]
@@ -50,9 +54,9 @@ constexpr int kBKEmpty = kBKFull + kPfStages;     // [kPfStages]
 constexpr int kBVFull = kBKEmpty + kPfStages;     // [kPfStages]
 constexpr int kBVEmpty = kBVFull + kPfStages;     // [kPfStages]
 constexpr int kBSFull = kBVEmpty + kPfStages;     // [2]
-constexpr int kBPFull = kBSFull + 2;              // [2], 128 arrivals
-constexpr int kBOFull = kBPFull + 2;              // [2], one per P buffer
-constexpr int kBDrain = kBOFull + 2;
+constexpr int kBPFull = kBSFull + 2;              // [key half][P buffer], 128 arrivals each
+constexpr int kBOFull = kBPFull + 4;              // [key half][P buffer]
+constexpr int kBDrain = kBOFull + 4;
 constexpr int kBNum = kBDrain + 1;
 
 // Shared memory: Q | K ring | V ring | P x 2 | barriers | misc.
@@ -62,8 +66,10 @@ constexpr int kOffV = kOffK + kPfStages * kPTile;
 constexpr int kOffP = kOffV + kPfStages * kPTile;
 constexpr int kOffBar = kOffP + 2 * kPTile;
 constexpr int kOffMisc = kOffBar + kBNum * 8;
-constexpr int kOffX = kOffMisc + 16;              // [2 halves][128 rows] floats: row maxima / sums
-constexpr int kPfSmem = kOffX + 2 * 128 * 4;
+constexpr int kPfSmem = kOffMisc + 16;
+// The final (m, l) exchange of the two halves ([2][2 halves][128 rows] floats) reuses the Q
+// tile: it happens after every product of the CTA has completed.
+constexpr int kOffX = kOffQ;
 constexpr size_t kPfSmemAlloc = (size_t)kPfSmem + 1024;   // + alignment slack
 
 // Named barrier 1 over the 256 softmax threads.
@@ -109,9 +115,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(bar(kBVFull + s), 1);
       mbar_init(bar(kBVEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kBSFull + s), 1);
-      mbar_init(bar(kBPFull + s), 256);
+    for (int s = 0; s < 2; ++s) mbar_init(bar(kBSFull + s), 1);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(bar(kBPFull + s), 128);
       mbar_init(bar(kBOFull + s), 1);
     }
     mbar_init(bar(kBDrain), 1);
@@ -188,12 +194,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       constexpr uint32_t kIdO = idesc_f16(128, 128, 0, 1);     // P K-major, V MN-major
       bool ok = mbar_wait(bar(kBQFull), 0, ctl);
       tc_fence_after();
-      int nqk = 0, npv = 0;
+      int nqk = 0, npv[2] = {0, 0};
       long long t_prog = now_ns();
       uint32_t spins = 0;
-      while (ok && npv < nk) {
+      while (ok && (npv[0] < nk || npv[1] < nk)) {
         bool prog = false;
-        if (nqk < nk && nqk <= npv + 1) {
+        // S(t) into buffer t & 1 once both halves have read S(t - 2) (their PV(t - 2) issued).
+        if (nqk < nk && nqk <= min(npv[0], npv[1]) + 1) {
           const int s = nqk % kPfStages;
           if (mbar_test(bar(kBKFull + s), (nqk / kPfStages) & 1)) {
             tc_fence_after();
@@ -211,23 +218,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             prog = true;
           }
         }
-        if (npv < nqk) {
-          const int s = npv % kPfStages;
-          if (mbar_test(bar(kBPFull + (npv & 1)), (npv >> 1) & 1) &&
-              mbar_test(bar(kBVFull + s), (npv / kPfStages) & 1)) {
-            tc_fence_after();
-            const uint32_t pb = sP + (npv & 1) * kPTile;
-            const uint32_t vb = sV + s * kPTile;
+        // O_h += P_h(t) V_h(t): P columns (keys) [64h, 64h + 64) times V rows [64h, 64h + 64).
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t pa = pb + (kk >> 2) * kPHalf + (kk & 3) * 32;
-              umma(tmem + kColO, sdesc(pa, 16, 1024, 2), sdesc(vb + kk * 2048, kPHalf, 1024, 2),
-                   kIdO, (npv > 0 || kk > 0) ? 1u : 0u);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int t = npv[hh];
+          if (t < nqk) {
+            const int s = t % kPfStages;
+            if (mbar_test(bar(kBPFull + 2 * hh + (t & 1)), (t >> 1) & 1) &&
+                mbar_test(bar(kBVFull + s), (t / kPfStages) & 1)) {
+              tc_fence_after();
+              const uint32_t pb = sP + (t & 1) * kPTile + hh * kPHalf;
+              const uint32_t vb = sV + s * kPTile + hh * 4 * 2048;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma(tmem + kColO + hh * 128, sdesc(pb + kk * 32, 16, 1024, 2),
+                     sdesc(vb + kk * 2048, kPHalf, 1024, 2), kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+              umma_commit(bar(kBOFull + 2 * hh + (t & 1)));
+              ++npv[hh];
+              // The V tile is free once both halves' products of it are issued.
+              if (npv[hh ^ 1] > t) umma_commit(bar(kBVEmpty + s));
+              prog = true;
             }
-            umma_commit(bar(kBOFull + (npv & 1)));
-            umma_commit(bar(kBVEmpty + s));
-            ++npv;
-            prog = true;
           }
         }
         if (prog) {
@@ -252,15 +263,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp >= 2 && warp <= 9) {
     // ------------------------------------------------------------------ softmax warps
     const int sub = warp & 3;
-    const int half = (warp - 2) >> 2;              // 64-column half of the tile (and of O)
+    const int half = (warp - 2) >> 2;              // key half of every tile
     const int r = 32 * sub + lane;                 // query row of this thread (TMEM lane)
     const int i = i0 + r;
     const int st = 128 * half + r;                 // softmax thread index 0..255
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * sub) << 16);
+    const uint32_t o_addr = lane_addr + kColO + 128 * half;   // this half's accumulator O_h
     const int lim = (i < Tb) ? min(Tb, (i / p.bs + 1) * p.bs) : 0;   // keys [0, lim)
     const float c2 = p.scale_log2;
-    float* xs = reinterpret_cast<float*>(base + kOffX);   // [2][128] half maxima, then sums
-    float m_ref = -INFINITY, l = 0.f;                       // l: this half's sum
+    float m_ref = -INFINITY, l = 0.f;              // this half's reference and row sum
     bool ok = true;
     for (int t = 0; t < nk; ++t) {
       const int j0 = t * kBN + 64 * half;          // first key of this thread's half
@@ -287,13 +298,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int u = 0; u < 8; ++u) mp[u] = x[u];
 #pragma unroll
       for (int e = 8; e < 64; ++e) mp[e & 7] = fmaxf(mp[e & 7], x[e]);
-      const float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      // The row's maximum from both halves (both threads of the row then take the same
-      // decisions below).
-      xs[st] = mh;
-      pf_bar();
-      float mt = fmaxf(mh, xs[st ^ 128]) * c2;    // log2 units (c2 > 0)
+      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * c2;
       // Lazy reference: raise it only when a score exceeds it by more than 2^8.
       const bool raise = mt > m_ref + kPfLazy || (m_ref == -INFINITY && mt > -INFINITY);
       float alpha = 1.f;
@@ -302,26 +308,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         l *= alpha;
         m_ref = mt;
       }
-      // Rows whose reference moved rescale their half of the O row (warp-uniform TMEM
-      // access), once the previous PV product is complete.
+      // Rows whose reference moved rescale their O_h row (warp-uniform TMEM access), once
+      // this half's previous PV product is complete.
       if (t > 0 && __any_sync(0xffffffffu, raise)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + 2 * half + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 64 / 16; ++c) {
+        for (int c = 0; c < 128 / 16; ++c) {
           float o[16];
-          const uint32_t col = kColO + 64 * half + 16 * c;
-          tmem_ld16(lane_addr + col, o);
+          tmem_ld16(o_addr + 16 * c, o);
           tc_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] *= alpha;
-          tmem_st16(lane_addr + col, o);
+          tmem_st16(o_addr + 16 * c, o);
         }
         tc_wait_st();
       }
-      // The P buffer of this tile was last read by the PV product two tiles ago.
+      // This half of the P buffer was last read by this half's PV product two tiles ago.
       if (t > 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + (t & 1)), ((t - 2) >> 1) & 1, ctl))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + 2 * half + (t & 1)), ((t - 2) >> 1) & 1, ctl))) { ok = false; break; }
         tc_fence_after();
       }
       // p = 2^(x c2 - m_ref), bf16 into this half of the swizzled K-major P row, 8 keys per
@@ -343,49 +348,60 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         store_p16(prow, 8 * half + k8, r, pk);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // Keys past the visible range in the last tile: zero their V rows so that 0 * x
-      // cannot become NaN in the product (those rows may hold anything).
+      // Keys of this half past the visible range (last tile): zero their V rows so that
+      // 0 * x cannot become NaN in the product (those rows may hold anything).
       const int valid = min(kBN, kmax - t * kBN);
-      if (valid < kBN) {
+      const int zlo = max(valid, 64 * half), zhi = 64 * half + 64;
+      if (zlo < zhi) {
         const int s = t % kPfStages;
         if (!__all_sync(0xffffffffu, mbar_wait(bar(kBVFull + s), (t / kPfStages) & 1, ctl))) { ok = false; break; }
         const uint32_t vbase = sV + s * kPTile;
-        for (int idx = st; idx < (kBN - valid) * 16; idx += 256) {
-          const int rr = valid + (idx >> 4), ch = idx & 15;
+        for (int idx = r; idx < (zhi - zlo) * 16; idx += 128) {
+          const int rr = zlo + (idx >> 4), ch = idx & 15;
           const uint32_t a = vbase + (ch >> 3) * kPHalf + rr * 128 + (ch & 7) * 16;
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(0u), "r"(0u),
                        "r"(0u), "r"(0u));
         }
       }
-      // Both halves have read the exchanged maxima before the next tile overwrites them.
-      pf_bar();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(kBPFull + (t & 1)));
+      mbar_arrive(bar(kBPFull + 2 * half + (t & 1)));
     }
-    // Epilogue: the row sum from both halves; each thread stores its 64 channels (128 bytes)
-    // of O / l as bf16.
+    // Epilogue: both halves' last products complete, then the pair merges
+    //   M = max(m_0, m_1), a_h = 2^(m_h - M), out = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1)
+    // and each thread stores 64 of the row's 128 channels (128 bytes) as bf16.
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBOFull + ((nk - 1) & 1)), ((nk - 1) >> 1) & 1, ctl));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBOFull + 2 + ((nk - 1) & 1)), ((nk - 1) >> 1) & 1, ctl));
     tc_fence_after();
-    xs[st] = l;
+    float* xs = reinterpret_cast<float*>(base + kOffX);   // [2 halves][128 rows] x (m, l)
+    xs[st] = m_ref;
+    xs[256 + st] = l;
     pf_bar();
-    const float lrow = l + xs[st ^ 128];
+    const float m0 = half ? xs[st ^ 128] : m_ref, m1 = half ? m_ref : xs[st ^ 128];
+    const float l0 = half ? xs[256 + (st ^ 128)] : l, l1 = half ? l : xs[256 + (st ^ 128)];
+    const float M = fmaxf(m0, m1);
+    const float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M);
+    const float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M);
+    const float L = a0 * l0 + a1 * l1;
+    const float inv = (ok && i < Tb && L > 0.f) ? 1.f / L : 0.f;
+    const float w0 = a0 * inv, w1 = a1 * inv;
     __nv_bfloat16* dst = p.out + (((size_t)b * p.T + i) * p.Hq + h) * kHeadDim + 64 * half;
-    const float inv = (ok && i < Tb && lrow > 0.f) ? 1.f / lrow : 0.f;
 #pragma unroll 1
     for (int c = 0; c < 64 / 16; ++c) {
-      float o[16];
+      float o0[16], o1[16];
       if (ok) {   // (warp-uniform)
-        tmem_ld16(lane_addr + kColO + 64 * half + 16 * c, o);
+        tmem_ld16(lane_addr + kColO + 64 * half + 16 * c, o0);
+        tmem_ld16(lane_addr + kColO + 128 + 64 * half + 16 * c, o1);
         tc_wait_ld();
       } else {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) o[e] = 0.f;
+        for (int e = 0; e < 16; ++e) o0[e] = o1[e] = 0.f;
       }
       uint32_t pk[8];
 #pragma unroll
       for (int e = 0; e < 16; e += 2) {
-        __nv_bfloat162 v2 = __floats2bfloat162_rn(o[e] * inv, o[e + 1] * inv);
+        __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(o0[e], w0, o1[e] * w1),
+                                                  fmaf(o0[e + 1], w0, o1[e + 1] * w1));
         pk[e >> 1] = *reinterpret_cast<uint32_t*>(&v2);
       }
       if (r < rows_here) {
