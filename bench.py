@@ -246,23 +246,47 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
         h_out = torch.empty_like(host["q"]).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in h_in.values())
         d2h = h_out.numel() * h_out.element_size()
-        for i in range(warmup):
-            d = dev[i % copies]
-            for n in h_in:
-                d[n].copy_(h_in[n], non_blocking=True)
-            one_step[i % copies].replay()
-            h_out.copy_(d["out"], non_blocking=True)
+        # Serving-loop pipelining: step i+1's inputs are copied in on a copy stream while step
+        # i computes, and step i's output is read back while step i+1 computes. Every step
+        # still moves its own inputs host -> device and its output device -> host inside the
+        # timed region; a buffer is reused only after the step that last used it finished.
+        comp_s, copy_s = torch.cuda.current_stream(), torch.cuda.Stream()
+        in_ready = [torch.cuda.Event() for _ in range(copies)]
+        done = [torch.cuda.Event() for _ in range(copies)]
+        used = [False] * copies
+
+        def upload(i):
+            k = i % copies
+            if used[k]:
+                copy_s.wait_event(done[k])
+            with torch.cuda.stream(copy_s):
+                for n in h_in:
+                    dev[k][n].copy_(h_in[n], non_blocking=True)
+            in_ready[k].record(copy_s)
+            used[k] = True
+
+        def run(n_steps):
+            upload(0)
+            for i in range(n_steps):
+                k = i % copies
+                comp_s.wait_event(in_ready[k])
+                one_step[k].replay()
+                done[k].record(comp_s)
+                if i + 1 < n_steps:
+                    upload(i + 1)
+                copy_s.wait_event(done[k])
+                with torch.cuda.stream(copy_s):
+                    h_out.copy_(dev[k]["out"], non_blocking=True)
+            comp_s.wait_stream(copy_s)
+
+        run(warmup)
         torch.cuda.synchronize()
         barrier()
+        used = [False] * copies
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for i in range(steps):
-            d = dev[i % copies]
-            for n in h_in:
-                d[n].copy_(h_in[n], non_blocking=True)
-            one_step[i % copies].replay()
-            h_out.copy_(d["out"], non_blocking=True)
-        e1.record()
+        e0.record(comp_s)
+        run(steps)
+        e1.record(comp_s)
         torch.cuda.synchronize()
         barrier()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1))
