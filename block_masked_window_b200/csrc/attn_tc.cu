@@ -805,10 +805,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (!mbar_wait(bar(kBarOFull + (glast & 1)), (glast >> 1) & 1, ctl)) { ok = false; break; }
       tc_fence_after();
 
-      // Epilogue: O^T row `row` (one channel) and the row sums (identical in every lane) are
-      // staged in the idle P^T buffer as [R][128] (bf16 output rows, or fp32 partial rows)
-      // and written by one asynchronous TMA store, so the warps do not stall on global
-      // stores while the memory system is saturated by the K/V stream.
+      // Epilogue: O^T row `row` (one channel) of a whole sequence is normalised, staged in the
+      // idle P^T buffer as [R][128] bf16 output rows and written by one TMA store; a partial
+      // is written straight to its slot.
       float* slot = sg.whole ? nullptr : slot_ptr(p, sg.slot);
       const uint32_t stg = sP;
       // Row sums: reduce the 128 key lanes' partials, 16 rows at a time. Within a warp a
@@ -871,7 +870,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                          "h"(*reinterpret_cast<const unsigned short*>(&v)));
           }
         }
+        fence_async_smem();
+        softmax_bar();
+        if (stid == 0) {
+          asm volatile(
+              "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                  reinterpret_cast<uint64_t>(&tmo)),
+              "r"(stg), "r"(0), "r"(sg.h * p.G), "r"(sg.b * p.W)
+              : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          // The staging buffer is reused as P^T by the next segment: wait until it was read.
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        }
       } else {
+        // A partial goes straight from registers to its slot: for each row the warp writes
+        // 32 consecutive channels (128 bytes), with no staging, barrier or copy to wait for.
+        float* accp = slot + 2 * p.rows_pad;
 #pragma unroll 1
         for (int c = 0; c < NQ / 16; ++c) {
           float ohi[16], olo[16];
@@ -882,33 +896,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int e = 0; e < 16; ++e) {
             const int q = 16 * c + e;
             if (q >= p.R) break;
-            asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + (uint32_t)(q * kHeadDim + row) * 4u),
-                         "f"(ohi[e] + olo[e]));
+            accp[(size_t)q * kHeadDim + row] = ohi[e] + olo[e];
           }
         }
-      }
-      if (!sg.whole && stid < p.R) {
-        slot[stid] = rowst[cur * NQ + stid];
-        slot[p.rows_pad + stid] = lsum[stid];
-      }
-      fence_async_smem();
-      softmax_bar();
-      if (stid == 0) {
-        if (sg.whole) {
-          asm volatile(
-              "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                  reinterpret_cast<uint64_t>(&tmo)),
-              "r"(stg), "r"(0), "r"(sg.h * p.G), "r"(sg.b * p.W)
-              : "memory");
-        } else {
-          asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                           slot + 2 * p.rows_pad),
-                       "r"(stg), "r"(p.R * kHeadDim * 4)
-                       : "memory");
+        if (stid < p.R) {
+          slot[stid] = rowst[cur * NQ + stid];
+          slot[p.rows_pad + stid] = lsum[stid];
         }
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        // The staging buffer is reused as P^T by the next segment: wait until it was read.
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       }
       // O, l and the shared per-segment buffers are reused by the next segment.
       tc_fence_before();
