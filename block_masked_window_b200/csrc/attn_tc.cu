@@ -36,6 +36,14 @@
 // threads as an MN-major, non-swizzled operand (8x8 core matrices: rows of 16 bytes, key
 // groups 128 bytes apart, row groups 2048 bytes apart), one 16-byte store per 8 rows.
 //
+// Options of the same kernel: the window append fused into the producers (la_pbd_step), key
+// limits per row (causal-window mask, per-sequence window lengths), and paged caches (a
+// template parameter, so that the contiguous kernels' code is unchanged). Before waiting for
+// the previous kernel of the stream, a small batch's first key tiles are prefetched into L2
+// from a guess of the plan. The epilogue stages a whole sequence's bf16 output rows in shared
+// memory for one TMA store; a split sequence's fp32 partial rows go straight from registers
+// to their slot.
+//
 // Every mbarrier wait is bounded: after ~2 s the CTA raises the sticky timeout flag in the
 // workspace header, the other roles stop at their next wait, in-flight copies and MMAs are
 // drained with bounded waits, TMEM is freed and the kernel returns.
