@@ -16,7 +16,8 @@ __all__ = [
     "LA_MASK_PBD", "LA_MASK_CAUSAL_WINDOW", "LA_ALGO_AUTO", "LA_ALGO_TCGEN05", "LA_ALGO_SIMT",
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
-    "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_attn_varwin",
+    "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
+    "la_pbd_attn_varwin",
     "la_pbd_step_varwin", "la_block_prefill", "la_pbd_attn_paged", "la_pbd_step_paged",
     "Workspace",
     "EXPORTED_SYMBOLS",
@@ -36,7 +37,7 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
 
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
-                    "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan",
+                    "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
                     "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill",
                     "la_pbd_attn_paged", "la_pbd_step_paged"]
 
@@ -112,7 +113,9 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_step_paged.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp,
                                       sz, vp]
     lib.la_pbd_plan.restype = i32
-    lib.la_pbd_plan.argtypes = [cfgp, i32, vp, i32, i32, vp, i32]
+    lib.la_pbd_plan.argtypes = [cfgp, i32, vp, i32, i32, i32, vp, i32]
+    lib.la_pbd_plan_params.restype = i32
+    lib.la_pbd_plan_params.argtypes = [i32, vp, vp]
     _LIB = lib
     return lib
 
@@ -256,21 +259,31 @@ def la_pbd_attn_static(cfg: Config, q, k_cache, v_cache, seq_lens, window_len: i
            "la_pbd_attn_static")
 
 
-def la_pbd_plan(cfg: Config, window_len: int, seq_lens, num_ctas: int, unit_keys: int):
+def la_pbd_plan(cfg: Config, window_len: int, seq_lens, num_ctas: int, unit_keys: int,
+                seg_units: int = 0):
     """Host-side split-KV work plan (no GPU work): a list of (cta, b, h, j0, j1, slot)
     tuples in CTA order; slot is -1 for a segment that is a whole sequence."""
     lens = (ctypes.c_int32 * cfg.batch)(*[int(x) for x in seq_lens])
     lib = load()
     n = lib.la_pbd_plan(ctypes.byref(cfg), int(window_len), ctypes.cast(lens, ctypes.c_void_p),
-                        int(num_ctas), int(unit_keys), None, 0)
+                        int(num_ctas), int(unit_keys), int(seg_units), None, 0)
     if n < 0:
         raise LaError(-n, "la_pbd_plan")
     buf = (ctypes.c_int32 * (6 * max(n, 1)))()
     m = lib.la_pbd_plan(ctypes.byref(cfg), int(window_len), ctypes.cast(lens, ctypes.c_void_p),
-                        int(num_ctas), int(unit_keys), ctypes.cast(buf, ctypes.c_void_p), n)
+                        int(num_ctas), int(unit_keys), int(seg_units),
+                        ctypes.cast(buf, ctypes.c_void_p), n)
     if m != n:
         raise LaError(LA_ERR_INVALID_ARG_CODE, "la_pbd_plan")
     return [tuple(buf[6 * i: 6 * i + 6]) for i in range(n)]
+
+
+def la_pbd_plan_params(algo: int):
+    """(unit_keys, seg_units) of the plan that attention kernel `algo` follows."""
+    unit, seg = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load().la_pbd_plan_params(int(algo), ctypes.byref(unit), ctypes.byref(seg)),
+           "la_pbd_plan_params")
+    return unit.value, seg.value
 
 
 def la_pbd_attn_varwin(cfg: Config, q, k_cache, v_cache, seq_lens, window_lens, window_max: int,

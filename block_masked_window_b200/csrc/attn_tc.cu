@@ -58,6 +58,7 @@ namespace {
 using namespace tc;
 
 constexpr int kNT = kTileKeys;          // 128 keys per tile
+constexpr int kSegUnits = 2;            // plan units charged per segment (tc_segment_units)
 constexpr int kKStages = 2;
 constexpr int kSBufs = 4;               // S^T buffers in TMEM: QK may run kSBufs-1 tiles ahead
 constexpr int kThreadsTc = 224;
@@ -334,7 +335,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const int P = __ldcg(p.seq_lens + lane);
       const int w = p.window_lens ? __ldcg(p.window_lens + lane) : p.W;
       const bool valid = P >= 0 && w >= 1 && w <= p.W && (long long)P + w <= (long long)p.S;
-      u = valid ? units_of(p, P + w) : 0;
+      u = valid ? plan_units_of(p, P + w) : 0;
     }
     int incl = u;
 #pragma unroll
@@ -352,11 +353,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int ub = __shfl_sync(0xffffffffu, u, bb), pb = __shfl_sync(0xffffffffu, excl, bb);
     if (lane == 0 && pos < Tg && starts != 0u && ub > 0) {
       const long long off = pos - (long long)p.Hkv * pb;
-      const int hh = (int)(off / ub), t0 = (int)(off - (long long)hh * ub);
+      const int hh = (int)(off / ub);
+      const int t0 = max((int)(off - (long long)hh * ub) - p.seg_units, 0);  // first key tile
       if (hh < p.Hkv) {
         tma_prefetch_3d(&tmq, 0, hh * p.G, bb * p.W);
         tma_prefetch_3d(&tmq, 64, hh * p.G, bb * p.W);
-        const int nt = (int)min((long long)(ub - t0), min(Cg, 2LL));
+        const int nt = (int)min((long long)(ub - p.seg_units - t0), min(Cg, 2LL));
         for (int t = 0; t < nt; ++t) {
           const int row = (bb * p.Hkv + hh) * p.S + (t0 + t) * kNT;
           tma_prefetch_2d(&tmk, 0, row);
@@ -931,6 +933,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
 int tc_ctas_per_sm() { return 1; }
 int tc_tile_keys() { return kNT; }
+// Fixed cost of a segment in tile times: a CTA pays it for each segment (Q load, the first
+// tile's exact-maximum pass, the epilogue, and the refill of the rings it leaves behind).
+int tc_segment_units() { return kSegUnits; }
 
 static int tc_nq(int R) { return round_up(R, 16); }
 

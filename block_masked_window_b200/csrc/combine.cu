@@ -36,7 +36,9 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
     const long long T0 = (long long)p.Hkv * p.pre_g[p.B];
     const long long C0 = plan_chunk(p, T0);
     const long long off0 = (long long)p.Hkv * p.pre_g[b] + (long long)h * u;
-    if (off0 / C0 != (off0 + u - 1) / C0) reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
+    int f0, l0;
+    plan_tile_ctas(p, off0, u, C0, &f0, &l0);
+    if (f0 != l0) reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
     return;
   }
   if (u == 0) {
@@ -47,7 +49,8 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
   const long long T = (long long)p.Hkv * p.pre_g[p.B];
   const long long C = plan_chunk(p, T);
   const long long off = (long long)p.Hkv * p.pre_g[b] + (long long)h * u;
-  const int c0 = (int)(off / C), c1 = (int)((off + u - 1) / C);
+  int c0, c1;
+  plan_tile_ctas(p, off, u, C, &c0, &c1);
   if (c0 == c1) return;
   const int ns = c1 - c0 + 1;
   const size_t stride = slot_floats(p.rows_pad);

@@ -89,7 +89,8 @@ la_status fill_problem(const la_pbd_cfg* cfg, int32_t W, Problem* p) {
 // Grid size: the resident capacity, but no more CTAs than the largest possible unit stream
 // (every sequence at full capacity) can keep busy at c_min units each.
 int grid_for(const Problem& p, int capacity) {
-  const long long max_units = (long long)p.B * p.Hkv * ((p.S + p.unit - 1) / p.unit);
+  const long long max_units =
+      (long long)p.B * p.Hkv * ((p.S + p.unit - 1) / p.unit + p.seg_units);
   const long long useful = (max_units + p.c_min - 1) / p.c_min;
   return (int)(useful < capacity ? (useful < 1 ? 1 : useful) : capacity);
 }
@@ -213,6 +214,7 @@ la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
     if (la::make_tma_maps(p, &maps, pool_rows) != cudaSuccess) return LA_ERR_CUDA;
     p.unit = la::tc_tile_keys();
     p.c_min = 1;
+    p.seg_units = la::tc_segment_units();
     p.num_ctas = grid_for(p, sms * la::tc_ctas_per_sm());
     e = la::launch_attn_tc(p, &maps.k, &maps.v, &maps.q, &maps.o, s);
   } else {
@@ -223,6 +225,7 @@ la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
     if (per_sm > la::kMaxCtasPerSm) per_sm = la::kMaxCtasPerSm;
     p.unit = la::simt_tile_keys();
     p.c_min = 1;
+    p.seg_units = 0;
     p.num_ctas = grid_for(p, sms * per_sm);
     e = la::launch_attn_simt(p, s);
   }
@@ -245,12 +248,26 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                      stream);
 }
 
+la_status la_pbd_plan_params(int32_t algo, int32_t* unit_keys, int32_t* seg_units) {
+  if (!unit_keys || !seg_units) return LA_ERR_INVALID_ARG;
+  if (algo == LA_ALGO_TCGEN05) {
+    *unit_keys = la::tc_tile_keys();
+    *seg_units = la::tc_segment_units();
+  } else if (algo == LA_ALGO_SIMT) {
+    *unit_keys = la::simt_tile_keys();
+    *seg_units = 0;
+  } else {
+    return LA_ERR_INVALID_ARG;
+  }
+  return LA_OK;
+}
+
 int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t W, const int32_t* seq_lens_host,
-                    int32_t num_ctas, int32_t unit_keys, int32_t* segments,
-                    int32_t max_segments) {
+                    int32_t num_ctas, int32_t unit_keys, int32_t seg_units,
+                    int32_t* segments, int32_t max_segments) {
   la_status st = check_cfg(cfg, W);
   if (st != LA_OK) return -(int32_t)st;
-  if (!seq_lens_host || num_ctas < 1 || unit_keys < 1 || max_segments < 0 ||
+  if (!seq_lens_host || num_ctas < 1 || unit_keys < 1 || seg_units < 0 || max_segments < 0 ||
       (max_segments > 0 && !segments))
     return -(int32_t)LA_ERR_INVALID_ARG;
   Problem p;
@@ -258,9 +275,10 @@ int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t W, const int32_t* seq_lens_ho
   p.seq_lens = seq_lens_host;
   p.unit = unit_keys;
   p.c_min = 1;
+  p.seg_units = seg_units;
   p.num_ctas = num_ctas;
   std::vector<int> pre(p.B + 1, 0);
-  for (int b = 0; b < p.B; ++b) pre[b + 1] = pre[b] + la::units_of(p, la::visible_len(p, b));
+  for (int b = 0; b < p.B; ++b) pre[b + 1] = pre[b] + la::plan_units_of(p, la::visible_len(p, b));
   const long long T = (long long)p.Hkv * pre[p.B];
   const long long C = la::plan_chunk(p, T);
   int32_t count = 0;

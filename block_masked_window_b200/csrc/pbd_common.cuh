@@ -53,7 +53,7 @@ struct Problem {
   __nv_bfloat16* vc;
   float* partials;              // slots, see slot_floats
   WsHeader* hdr;
-  int* pre_g;                   // [B+1] prefix sums of U_b, written by attention CTA 0
+  int* pre_g;                   // [B+1] prefix sums of plan units, written by attention CTA 0
   int B, Hq, Hkv, G, W, S;      // G = Hq / Hkv; W = the (longest) window length
   int R;                        // rows per sequence = W * G
   int rows_pad;                 // R rounded up to 16: rows per partial slot
@@ -61,6 +61,7 @@ struct Problem {
   int num_ctas;                 // grid size of the attention kernel (fixes the chunk size)
   int unit;                     // keys per plan unit (the attention kernel's key tile)
   int c_min;                    // minimum units per CTA
+  int seg_units;                // plan units charged per (sequence, KV head) besides its tiles
   float scale_log2;             // scale * log2(e)
 };
 
@@ -110,10 +111,20 @@ __host__ __device__ inline int visible_len(const Problem& p, int b) {
   return P + w;
 }
 
-// Plan units of sequence b.
+// Key tiles of a sequence with n visible keys.
 __host__ __device__ inline int units_of(const Problem& p, int n) { return (n + p.unit - 1) / p.unit; }
 
-// Block-wide prefix sum of U_b into pre[0..B] (pre[0] = 0, pre[b+1] = U_0 + ... + U_b).
+// Plan units of one (sequence, KV head) with n visible keys: seg_units units that stand for
+// the fixed cost of a segment (loading Q, the first tile's exact maximum, the epilogue),
+// followed by one unit per key tile. Charging the fixed cost in the plan gives a CTA whose
+// run crosses sequence starts fewer tiles, so that CTAs with several segments do not finish
+// last. An invalid sequence (n = 0) has no units.
+__host__ __device__ inline int plan_units_of(const Problem& p, int n) {
+  return n > 0 ? units_of(p, n) + p.seg_units : 0;
+}
+
+// Block-wide prefix sum of the plan units U_b (plan_units_of) into pre[0..B] (pre[0] = 0,
+// pre[b+1] = U_0 + ... + U_b).
 // Every thread of the block must call it. `warp_tot` needs one int per warp (<= 32).
 __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
   const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, wid = tid >> 5;
@@ -122,7 +133,7 @@ __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
   if (tid == 0) pre[0] = 0;
   for (int base = 0; base < p.B; base += nthr) {
     int b = base + tid;
-    int x = (b < p.B) ? units_of(p, visible_len(p, b)) : 0;
+    int x = (b < p.B) ? plan_units_of(p, visible_len(p, b)) : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -172,7 +183,10 @@ struct Segment {
   int slot;        // partial slot (when !whole)
 };
 
-// Iterator over the segments of CTA `c`.
+// Iterator over the segments of CTA `c`. The units of (b, h) start at s0: seg_units fixed-cost
+// units, then its key tiles from t0 = s0 + seg_units on. A CTA whose run holds only fixed-cost
+// units of (b, h) gets no segment of it; the CTA holding tile 0 does the sequence's first
+// segment.
 struct SegmentIter {
   long long pos, end;
   int b, h;
@@ -184,20 +198,32 @@ struct SegmentIter {
         if (++h == p.Hkv) { h = 0; ++b; }
         continue;
       }
-      long long lo = pos, hi = (end < s0 + u) ? end : s0 + u;
+      const long long t0 = s0 + p.seg_units;
+      const long long hi = (end < s0 + u) ? end : s0 + u;
+      const long long lo = pos > t0 ? pos : t0;
+      pos = hi;
+      if (hi <= t0) continue;  // only fixed-cost units of (b, h) in this CTA
       const int n = visible_len(p, b);
       sg.b = b; sg.h = h; sg.n = n; sg.w = window_of(p, b);
-      sg.j0 = (int)(lo - s0) * p.unit;
-      const int e = (int)(hi - s0) * p.unit;
+      sg.j0 = (int)(lo - t0) * p.unit;
+      const int e = (int)(hi - t0) * p.unit;
       sg.j1 = e < n ? e : n;
-      sg.whole = (lo == s0 && hi == s0 + u);
+      sg.whole = (lo == t0 && hi == s0 + u);
       sg.slot = c + b * p.Hkv + h;
-      pos = hi;
       return true;
     }
     return false;
   }
 };
+
+// CTAs that hold the first and the last key tile of (b, h), whose units start at s0 = off
+// and number u > 0 (chunk size C): the sequence is split iff they differ, and its partial
+// results sit in slots c + b * Hkv + h for c in [first, last].
+__host__ __device__ inline void plan_tile_ctas(const Problem& p, long long off, int u, long long C,
+                                               int* first, int* last) {
+  *first = (int)((off + p.seg_units) / C);
+  *last = (int)((off + u - 1) / C);
+}
 
 __host__ __device__ inline SegmentIter plan_begin(const Problem& p, const int* pre, int c, long long C,
                                          long long T) {

@@ -28,6 +28,7 @@ struct TmaMaps {
 
 int tc_ctas_per_sm();
 int tc_tile_keys();
+int tc_segment_units();
 
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

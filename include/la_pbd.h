@@ -234,10 +234,13 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
 /*
  * Host-side view of the split-KV work plan that la_pbd_attn follows on the device, for
  * inspection and testing; touches no GPU. The keys [0, P_b + W) of each (sequence b, KV
- * head h) are cut into units of `unit_keys` keys (the attention kernel's key tile: 128 for
- * the tcgen05 kernel, 32 for the CUDA-core kernel), all units are laid end to end, and CTA c
- * of `num_ctas` takes one contiguous run of them; the part of a (b, h) in one CTA is a
- * segment. Sequences with an invalid prefix length contribute nothing.
+ * head h) are cut into tiles of `unit_keys` keys (the attention kernel's key tile), and
+ * (b, h) occupies `seg_units` units standing for the fixed cost of a segment followed by one
+ * unit per tile. All units are laid end to end, and CTA c of `num_ctas` takes one
+ * contiguous run of them; the tiles of a (b, h) in one CTA are a segment (a CTA whose run
+ * holds only fixed-cost units of (b, h) gets none of it). The attention kernels use
+ * unit_keys = 128, seg_units = 2 (tcgen05 kernel) and unit_keys = 32, seg_units = 0
+ * (CUDA-core kernel). Sequences with an invalid prefix length contribute nothing.
  *   seq_lens_host  host int32 [cfg->batch]
  *   segments       host int32 [max_segments][6], written in CTA order as
  *                  {cta, b, h, j0, j1, slot}: keys [j0, j1) of (b, h); slot = -1 when the
@@ -245,11 +248,18 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
  *                  workspace slot of its partial result
  * Returns the number of segments (which may exceed max_segments; only the first
  * max_segments are written), or -la_status on invalid arguments (num_ctas < 1,
- * unit_keys < 1, a null pointer, an invalid cfg).
+ * unit_keys < 1, seg_units < 0, a null pointer, an invalid cfg).
  */
 int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t window_len, const int32_t* seq_lens_host,
-                    int32_t num_ctas, int32_t unit_keys, int32_t* segments,
+                    int32_t num_ctas, int32_t unit_keys, int32_t seg_units, int32_t* segments,
                     int32_t max_segments);
+
+/*
+ * The plan parameters that an attention kernel uses: its key tile (`*unit_keys`) and the
+ * fixed segment cost in tiles (`*seg_units`), for algo LA_ALGO_TCGEN05 or LA_ALGO_SIMT.
+ * Host only. LA_ERR_INVALID_ARG for another algo or a null pointer.
+ */
+la_status la_pbd_plan_params(int32_t algo, int32_t* unit_keys, int32_t* seg_units);
 
 /*
  * Synchronise `stream`, read and clear the workspace's sticky device-side error flags.

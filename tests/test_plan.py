@@ -3,10 +3,14 @@ kernels run on the device, evaluated on the host).
 
 The plan must cover the visible keys [0, P_b + W) of every (sequence, KV head) exactly once,
 in whole key tiles (only a sequence's last tile may be short, and no tile is shared by two
-CTAs), give every CTA at most its share of tiles, mark a segment as whole exactly when it is
-the only segment of its sequence, and hand partial segments distinct workspace slots below
-num_ctas + B * Hkv (the slot count the workspace is sized for)."""
+CTAs), give every CTA at most its share of plan units (its tiles, plus the fixed segment cost
+of every segment after its first, which starts a sequence inside the CTA's run), mark a
+segment as whole exactly when it is the only segment of its sequence, and hand partial
+segments distinct workspace slots below num_ctas + B * Hkv (the slot count the workspace is
+sized for)."""
 import random
+
+import torch
 
 import pytest
 
@@ -20,14 +24,14 @@ def _built():
     bmw.load()
 
 
-def check_plan(seq_lens, W, S, Hkv, num_ctas, unit, Hq=None):
+def check_plan(seq_lens, W, S, Hkv, num_ctas, unit, Hq=None, seg=0):
     Hq = Hq or 8 * Hkv
     cfg = bmw.Config.make(len(seq_lens), Hq, Hkv, S)
-    segs = bmw.la_pbd_plan(cfg, W, seq_lens, num_ctas, unit)
+    segs = bmw.la_pbd_plan(cfg, W, seq_lens, num_ctas, unit, seg)
     B = len(seq_lens)
     valid = [0 <= P and P + W <= S for P in seq_lens]
     n_of = [P + W if ok else 0 for P, ok in zip(seq_lens, valid)]
-    units = sum(Hkv * -(-n // unit) for n in n_of)
+    units = sum(Hkv * (-(-n // unit) + seg) for n in n_of if n > 0)
     C = max(1, -(-units // num_ctas))
 
     covered = {}
@@ -45,14 +49,19 @@ def check_plan(seq_lens, W, S, Hkv, num_ctas, unit, Hq=None):
         assert j0 % unit == 0, "segments start on a tile boundary"
         assert j1 % unit == 0 or j1 == n, "segments end on a tile boundary or at the end"
         covered.setdefault((b, h), []).append((j0, j1, cta, slot))
-        per_cta_units[cta] = per_cta_units.get(cta, 0) + -(-(j1 - j0) // unit)
+        # a segment after the CTA's first starts its sequence inside the run: its fixed cost
+        # units are in the run too
+        fixed = seg if cta in per_cta_units else 0
+        if fixed:
+            assert j0 == 0, "only a CTA's first segment may continue a sequence"
+        per_cta_units[cta] = per_cta_units.get(cta, 0) + fixed + -(-(j1 - j0) // unit)
         if slot != -1:
             assert slot not in slots, "partial slots must be distinct"
             assert 0 <= slot < num_ctas + B * Hkv
             slots.add(slot)
 
     for cta, u in per_cta_units.items():
-        assert u <= C, f"CTA {cta} got {u} tiles, share is {C}"
+        assert u <= C, f"CTA {cta} got {u} units, share is {C}"
     for b in range(B):
         for h in range(Hkv):
             parts = sorted(covered.get((b, h), []))
@@ -71,11 +80,12 @@ def check_plan(seq_lens, W, S, Hkv, num_ctas, unit, Hq=None):
     return segs
 
 
+@pytest.mark.parametrize("seg", [0, 2, 5])
 @pytest.mark.parametrize("unit", [128, 32])
 @pytest.mark.parametrize("num_ctas", [1, 7, 17, 148, 592])
-def test_plan_single_image_and_long(unit, num_ctas):
-    check_plan([1024], 6, 1088, 2, num_ctas, unit)
-    check_plan([32768] * 8, 6, 32832, 2, num_ctas, unit)
+def test_plan_single_image_and_long(unit, num_ctas, seg):
+    check_plan([1024], 6, 1088, 2, num_ctas, unit, seg=seg)
+    check_plan([32768] * 8, 6, 32832, 2, num_ctas, unit, seg=seg)
 
 
 @pytest.mark.parametrize("seed", range(6))
@@ -87,24 +97,61 @@ def test_plan_ragged(seed):
     lens = [rng.randint(0, S - W) for _ in range(B)]
     for num_ctas in (1, 13, 148, 592):
         for unit in (128, 32):
-            check_plan(lens, W, S, 2, num_ctas, unit)
+            for seg in (0, 1, 2, 3):
+                check_plan(lens, W, S, 2, num_ctas, unit, seg=seg)
+
+
+def test_plan_params():
+    assert bmw.la_pbd_plan_params(bmw.LA_ALGO_TCGEN05) == (128, 2)
+    assert bmw.la_pbd_plan_params(bmw.LA_ALGO_SIMT) == (32, 0)
+    with pytest.raises(bmw.LaError):
+        bmw.la_pbd_plan_params(bmw.LA_ALGO_AUTO)
+
+
+def cta_costs(segs, seg):
+    """Cost of each CTA in tile times: its tiles plus `seg` for each of its segments."""
+    cost = {}
+    for cta, b, h, j0, j1, slot in segs:
+        cost[cta] = cost.get(cta, 0) + seg + -(-(j1 - j0) // 128)
+    return cost
+
+
+def test_plan_fixed_cost_balances_ragged_batch():
+    """The 64-sequence ragged batch (prefixes U{512..4096} + U{1..5}, window 6): with the
+    fixed segment cost in the plan, the costliest CTA (tiles + 2 per segment) is cheaper than
+    with a plan of tiles only, where CTAs that cross several sequence starts finish last."""
+    gen = torch.Generator().manual_seed(3)
+    base = torch.randint(512, 4096 + 1, (64,), generator=gen, dtype=torch.int64)
+    acc = torch.randint(1, 5 + 1, (64,), generator=gen, dtype=torch.int64)
+    lens = (base + acc).tolist()
+    unit, seg = bmw.la_pbd_plan_params(bmw.LA_ALGO_TCGEN05)
+    flat = check_plan(lens, 6, 4160, 2, 148, unit, seg=0)
+    fixed = check_plan(lens, 6, 4160, 2, 148, unit, seg=seg)
+    worst_flat = max(cta_costs(flat, seg).values())
+    worst_fixed = max(cta_costs(fixed, seg).values())
+    assert worst_fixed < worst_flat, (worst_fixed, worst_flat)
 
 
 def test_plan_edge_cases():
     # empty prefixes, exact tile multiples, invalid lengths, one head
-    check_plan([0, 0, 0], 6, 64, 2, 5, 128)
-    check_plan([122, 250, 506], 6, 512, 2, 3, 128)       # P + W = 128, 256, 512
-    check_plan([-1, 100, 60, 59], 6, 66, 2, 4, 32)       # P = -1 and P = 100 are invalid
-    check_plan([5, 7], 1, 8, 1, 2, 128, Hq=16)
+    for seg in (0, 2):
+        check_plan([0, 0, 0], 6, 64, 2, 5, 128, seg=seg)
+        check_plan([122, 250, 506], 6, 512, 2, 3, 128, seg=seg)    # P + W = 128, 256, 512
+        check_plan([-1, 100, 60, 59], 6, 66, 2, 4, 32, seg=seg)    # P = -1, 100 invalid
+        check_plan([5, 7], 1, 8, 1, 2, 128, Hq=16, seg=seg)
     segs = check_plan([1024], 6, 1088, 2, 18, 128)
     # single-image decode at one tile per CTA: 9 tiles per KV head, every CTA one segment
     assert len(segs) == 18 and len({s[0] for s in segs}) == 18
+    # with the fixed cost, 22 units at one per CTA: each KV head's two fixed-cost units
+    # fall in CTAs of their own, which get no segment; the 18 tiles still go one per CTA
+    segs = check_plan([1024], 6, 1088, 2, 22, 128, seg=2)
+    assert sorted(s[0] for s in segs) == list(range(2, 11)) + list(range(13, 22))
 
 
 def test_plan_rejects_bad_arguments():
     cfg = bmw.Config.make(2, 16, 2, 128)
-    for num_ctas, unit in ((0, 128), (4, 0)):
+    for num_ctas, unit, seg in ((0, 128, 0), (4, 0, 0), (4, 128, -1)):
         with pytest.raises(bmw.LaError):
-            bmw.la_pbd_plan(cfg, 6, [1, 2], num_ctas, unit)
+            bmw.la_pbd_plan(cfg, 6, [1, 2], num_ctas, unit, seg)
     with pytest.raises(bmw.LaError):
         bmw.la_pbd_plan(bmw.Config.make(2, 16, 3, 128), 6, [1, 2], 4, 128)
