@@ -460,6 +460,7 @@ def main():
             "attn_launch_us": r["launch_us"], "attn_bytes_per_launch": r["alg_bytes"],
             "achieved_gbs": r["achieved_gbs"], "frac_of_measured_hbm": r["achieved_gbs"] / peak,
             "frac_of_8tbs": r["achieved_gbs"] / 8000.0,
+            "traffic": stored_traffic(name),
         })
 
     prefill = None if args.no_prefill else measure_prefill(args, device, bmw, torch, barrier,
