@@ -214,8 +214,14 @@ la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
     if (la::make_tma_maps(p, &maps, pool_rows) != cudaSuccess) return LA_ERR_CUDA;
     p.unit = la::tc_tile_keys();
     p.c_min = 1;
-    p.seg_units = la::tc_segment_units();
-    p.num_ctas = grid_for(p, sms * la::tc_ctas_per_sm());
+    p.seg_units = 0;
+    const int cap = sms * la::tc_ctas_per_sm();
+    // The fixed segment cost only matters when a CTA can get several tiles. When even full
+    // caches have no more tiles than the grid has CTAs, every CTA gets at most one tile, and
+    // the cost would only add CTAs without work.
+    if ((long long)p.B * p.Hkv * ((p.S + p.unit - 1) / p.unit) > cap)
+      p.seg_units = la::tc_segment_units();
+    p.num_ctas = grid_for(p, cap);
     e = la::launch_attn_tc(p, &maps.k, &maps.v, &maps.q, &maps.o, s);
   } else {
     int per_sm = 0;

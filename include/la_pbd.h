@@ -240,7 +240,9 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
  * contiguous run of them; the tiles of a (b, h) in one CTA are a segment (a CTA whose run
  * holds only fixed-cost units of (b, h) gets none of it). The attention kernels use
  * unit_keys = 128, seg_units = 2 (tcgen05 kernel) and unit_keys = 32, seg_units = 0
- * (CUDA-core kernel). Sequences with an invalid prefix length contribute nothing.
+ * (CUDA-core kernel); the tcgen05 kernel uses seg_units = 0 when B * Hkv * ceil(S_max / 128)
+ * does not exceed its grid (148 CTAs on B200), where every CTA gets at most one tile.
+ * Sequences with an invalid prefix length contribute nothing.
  *   seq_lens_host  host int32 [cfg->batch]
  *   segments       host int32 [max_segments][6], written in CTA order as
  *                  {cta, b, h, j0, j1, slot}: keys [j0, j1) of (b, h); slot = -1 when the
@@ -256,7 +258,8 @@ int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t window_len, const int32_t* se
 
 /*
  * The plan parameters that an attention kernel uses: its key tile (`*unit_keys`) and the
- * fixed segment cost in tiles (`*seg_units`), for algo LA_ALGO_TCGEN05 or LA_ALGO_SIMT.
+ * fixed segment cost in tiles (`*seg_units`; applied only when a CTA can get several
+ * tiles, see la_pbd_plan), for algo LA_ALGO_TCGEN05 or LA_ALGO_SIMT.
  * Host only. LA_ERR_INVALID_ARG for another algo or a null pointer.
  */
 la_status la_pbd_plan_params(int32_t algo, int32_t* unit_keys, int32_t* seg_units);

@@ -118,6 +118,26 @@ def test_many_short_sequences(algo):
     assert_parity(gpu, ref, "300 short sequences")
 
 
+def test_plan_fixed_cost_shapes():
+    """34 sequences of 1-3 key tiles in a 1024-row cache: the tcgen05 plan charges each
+    (sequence, KV head) two fixed-cost units, so with two units per CTA some CTAs hold only
+    fixed-cost units (no segment), some start inside them, and the rest split sequences or
+    own them whole. The host view of the same plan confirms that the case has all three."""
+    rng = np.random.default_rng(0)
+    prefixes = tuple(int(x) for x in rng.integers(0, 380, size=34))
+    wi = workloads.random_case(34, prefixes, 6, seed=21, max_seq=1024)
+    unit, seg = bmw.la_pbd_plan_params(bmw.LA_ALGO_TCGEN05)
+    cfg = bmw.Config.make(34, 16, 2, 1024)
+    plan = bmw.la_pbd_plan(cfg, 6, prefixes, 148, unit, seg)
+    used = {c for c, *_ in plan}
+    assert len(used) < max(used) + 1, "some CTA holds only fixed-cost units"
+    assert any(slot >= 0 for *_, slot in plan) and any(slot < 0 for *_, slot in plan)
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=bmw.LA_ALGO_TCGEN05)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(gpu, ref, "fixed-cost plan shapes")
+
+
 @pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
 def test_invalid_prefix_lengths_flagged(algo):
     """P < 0 or P + W > max_seq: zero output rows, untouched cache, sticky status."""
