@@ -221,6 +221,17 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
     ms_per_step = ms / (replays * inner)
     value = aggregate_throughput(world, B, replays * inner, ms)
 
+    # Launch floor: a graph of as many empty kernels as one replay of the step graph launches
+    # (programmatic dependent launch, one CTA of 224 threads per SM), timed the same way.
+    per_step_launches = L * (2 if uses_tc else 3)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    floor_graph = capture(torch, lambda: bmw.la_noop_chain(inner * per_step_launches, sms, 224))
+    ms_floor = max_over_ranks(time_graphs(torch, [floor_graph], replays, warmup, barrier))
+    launch_floor = {"ms_per_step": ms_floor / (replays * inner),
+                    "launches_per_step": per_step_launches,
+                    "kernel": f"empty, programmatic dependent launch, {sms} CTAs x 224 threads"}
+    del floor_graph
+
     # Dominant kernel: the attention call of one layer (attention + split merge), timed alone
     # over the same rotating copies.
     attn_graphs = [capture(torch, lambda ds=seq_of(i): [run_attn_only(bmw, cfg, d, seq, W, ws, L) for d in ds])
@@ -301,7 +312,7 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
         "step_bytes": step_bytes, "copies": copies, "e2e": e2e, "layers": L,
         # per layer: attention (with the append fused in on the tcgen05 path) + merge; the
         # CUDA-core path runs the append kernel too
-        "launches_per_step": L * (2 if uses_tc else 3),
+        "launches_per_step": per_step_launches, "launch_floor": launch_floor,
     }
 
 
@@ -458,6 +469,7 @@ def main():
             "batch": swl.batch, "window": swl.window, "layers": swl.layers,
             "window_steps_per_s": r["value"], "ms_per_step": r["ms_per_step"],
             "attn_launch_us": r["launch_us"], "attn_bytes_per_launch": r["alg_bytes"],
+            "launch_floor_ms_per_step": r["launch_floor"]["ms_per_step"],
             "achieved_gbs": r["achieved_gbs"], "frac_of_measured_hbm": r["achieved_gbs"] / peak,
             "frac_of_8tbs": r["achieved_gbs"] / 8000.0,
             "traffic": stored_traffic(name),
@@ -488,6 +500,7 @@ def main():
                      "bytes_per_launch": res["alg_bytes"], "launch_us": res["launch_us"]},
         "gpu_launches": res["launches_per_step"] * args.steps,
         "e2e": res["e2e"], "clocks": res["clocks"], "cpu_baseline": cb,
+        "launch_floor": res["launch_floor"],
         "step_bytes": res["step_bytes"],
         "step_gbs": res["step_bytes"] / (res["ms_per_step"] * 1e-3) / 1e9,
         "sweep": sweep,

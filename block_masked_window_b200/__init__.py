@@ -17,7 +17,7 @@ __all__ = [
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
     "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
-    "la_pbd_attn_varwin",
+    "la_noop_chain", "la_pbd_attn_varwin",
     "la_pbd_step_varwin", "la_block_prefill", "la_pbd_attn_paged", "la_pbd_step_paged",
     "Workspace",
     "EXPORTED_SYMBOLS",
@@ -38,6 +38,7 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
                     "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
+                    "la_noop_chain",
                     "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill",
                     "la_pbd_attn_paged", "la_pbd_step_paged"]
 
@@ -116,6 +117,8 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_plan.argtypes = [cfgp, i32, vp, i32, i32, i32, vp, i32]
     lib.la_pbd_plan_params.restype = i32
     lib.la_pbd_plan_params.argtypes = [i32, vp, vp]
+    lib.la_noop_chain.restype = i32
+    lib.la_noop_chain.argtypes = [i32, i32, i32, vp]
     _LIB = lib
     return lib
 
@@ -276,6 +279,12 @@ def la_pbd_plan(cfg: Config, window_len: int, seq_lens, num_ctas: int, unit_keys
     if m != n:
         raise LaError(LA_ERR_INVALID_ARG_CODE, "la_pbd_plan")
     return [tuple(buf[6 * i: 6 * i + 6]) for i in range(n)]
+
+
+def la_noop_chain(launches: int, ctas: int, threads: int, stream=None) -> None:
+    """Enqueue `launches` empty kernels (launch-floor measurements)."""
+    _check(load().la_noop_chain(int(launches), int(ctas), int(threads), _stream(stream)),
+           "la_noop_chain")
 
 
 def la_pbd_plan_params(algo: int):

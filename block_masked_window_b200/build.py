@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libla_pbd.so")
 SOURCES = ["la_pbd_api.cu", "kv_append.cu", "attn_simt.cu", "attn_tc.cu", "combine.cu",
-           "la_pbd_static.cu", "prefill_tc.cu"]
+           "la_pbd_static.cu", "prefill_tc.cu", "noop.cu"]
 
 
 def nvcc() -> str:

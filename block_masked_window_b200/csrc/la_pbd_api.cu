@@ -254,6 +254,13 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                      stream);
 }
 
+la_status la_noop_chain(int32_t launches, int32_t ctas, int32_t threads, void* stream) {
+  if (launches < 0 || ctas < 1 || threads < 1 || threads > 1024) return LA_ERR_INVALID_ARG;
+  for (int i = 0; i < launches; ++i)
+    if (la::launch_noop(ctas, threads, (cudaStream_t)stream) != cudaSuccess) return LA_ERR_CUDA;
+  return LA_OK;
+}
+
 la_status la_pbd_plan_params(int32_t algo, int32_t* unit_keys, int32_t* seg_units) {
   if (!unit_keys || !seg_units) return LA_ERR_INVALID_ARG;
   if (algo == LA_ALGO_TCGEN05) {

@@ -29,6 +29,9 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, void* k_cache
                              const int32_t* seq_lens, const int32_t* window_lens, int B, int W,
                              int Hkv, int S, cudaStream_t stream);
 
+// Empty kernel with programmatic dependent launch (launch-floor measurements).
+cudaError_t launch_noop(int ctas, int threads, cudaStream_t stream);
+
 // CUDA-core split-KV attention (any R = W * G <= 128).
 int simt_rows_per_thread(int R);
 int simt_tile_keys();

@@ -257,6 +257,15 @@ int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t window_len, const int32_t* se
                     int32_t max_segments);
 
 /*
+ * Launch-floor helper: enqueue `launches` empty kernels of `ctas` x `threads` on `stream`,
+ * chained with programmatic dependent launch like the library's own kernels. Timing a CUDA
+ * graph of these beside a graph of real calls with the same launch count gives the part of
+ * the step that launching alone costs. Asynchronous; allocates nothing. LA_ERR_INVALID_ARG
+ * for launches < 0, ctas < 1 or threads outside [1, 1024]; LA_ERR_CUDA if a launch fails.
+ */
+la_status la_noop_chain(int32_t launches, int32_t ctas, int32_t threads, void* stream);
+
+/*
  * The plan parameters that an attention kernel uses: its key tile (`*unit_keys`) and the
  * fixed segment cost in tiles (`*seg_units`; applied only when a CTA can get several
  * tiles, see la_pbd_plan), for algo LA_ALGO_TCGEN05 or LA_ALGO_SIMT.

@@ -98,3 +98,12 @@ def test_binding_rejects_cpu_tensors(lib):
         bmw.la_kv_append(cfg, q[:, :, :2], q[:, :, :2], torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16),
                          torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16),
                          torch.zeros(1, dtype=torch.int32), 6)
+
+
+def test_noop_chain_validates_before_launching(lib):
+    # every one of these is rejected on the host, before any CUDA call
+    assert lib.la_noop_chain(-1, 1, 32, None) == 1
+    assert lib.la_noop_chain(4, 0, 32, None) == 1
+    assert lib.la_noop_chain(4, 1, 0, None) == 1
+    assert lib.la_noop_chain(4, 1, 1025, None) == 1
+    assert lib.la_noop_chain(0, 1, 32, None) == 0     # nothing to launch
