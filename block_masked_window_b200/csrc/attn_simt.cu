@@ -116,8 +116,8 @@ __global__ void __launch_bounds__(kThreads) pbd_attn_simt_kernel(Problem p) {
   constexpr int ROWS = 16 * RPT;
   constexpr int PROWS = 2 * RPT;  // rows per thread in the PV phase
 
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();   // after the wait: the merge kernel reads seq_lens before its own wait
   plan_prefix(p, s.pre, s.warp_tot);
   __syncthreads();
   const long long T = (long long)p.Hkv * s.pre[p.B];

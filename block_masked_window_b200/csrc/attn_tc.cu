@@ -283,7 +283,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Ctl ctl{abort_flag, p.hdr};
-  pdl_trigger();
   if (tid == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
@@ -334,8 +333,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (lane < p.B) {
       const int P = __ldcg(p.seq_lens + lane);
       const int w = p.window_lens ? __ldcg(p.window_lens + lane) : p.W;
-      const bool valid = P >= 0 && w >= 1 && w <= p.W && (long long)P + w <= (long long)p.S;
-      u = valid ? plan_units_of(p, P + w) : 0;
+      u = plan_units_of(p, visible_of(p, P, w));
     }
     int incl = u;
 #pragma unroll
@@ -370,8 +368,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   }
   // Everything above is on-chip (or an L2 hint); from here on global memory written by the
-  // previous kernel of the stream is read.
+  // previous kernel of the stream is read. The merge kernel after this one may start only
+  // once every CTA is past the wait (it reads seq_lens before its own wait).
   pdl_wait();
+  pdl_trigger();
   plan_prefix(p, pre, warp_tot);
   fence_async_smem();
   tc_fence_before();

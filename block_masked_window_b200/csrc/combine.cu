@@ -22,22 +22,53 @@ constexpr int kMerge = 16;               // partials loaded in the first round t
 __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem p) {
   __shared__ float s_w[kCombineRows][kCombineMaxSlots];
   pdl_trigger();
-  pdl_wait();
   const int s = blockIdx.y;            // sequence = b * Hkv + h
   const int b = s / p.Hkv, h = s - b * p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * kCombineRows + warp;
-  const int u = p.pre_g[b + 1] - p.pre_g[b];   // plan units of the sequence
+  // The plan of sequence b: its units u, the units pb before it and the total. For a batch of
+  // up to 32 sequences each warp derives it before the dependency wait from seq_lens and
+  // window_lens (L2 reads; the attention kernel before this one does not write them, and it
+  // lets this kernel start only after its own wait, so their last writer has completed).
+  // After the wait only the partials remain to be read. A larger batch reads the prefix
+  // sums that attention CTA 0 published.
+  int u = 0, pb = 0, ptot = 0, wb = p.W;
+  const bool small = p.B <= 32;
+  if (small) {
+    int x = 0, w = p.W;
+    if (lane < p.B) {
+      const int P = __ldcg(p.seq_lens + lane);
+      if (p.window_lens) w = __ldcg(p.window_lens + lane);
+      x = plan_units_of(p, visible_of(p, P, w));
+    }
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    u = __shfl_sync(0xffffffffu, x, b);
+    pb = __shfl_sync(0xffffffffu, incl - x, b);
+    wb = __shfl_sync(0xffffffffu, w, b);
+    ptot = __shfl_sync(0xffffffffu, incl, 31);
+  }
+  pdl_wait();
+  if (!small) {
+    pb = p.pre_g[b];
+    u = p.pre_g[b + 1] - pb;
+    ptot = p.pre_g[p.B];
+    wb = window_of(p, b);
+  }
   if (r >= p.R) return;
   __nv_bfloat16* dst = p.out + out_row_offset(p, b, h, r);
-  if (u > 0 && r / p.G >= window_of(p, b)) {
+  const long long T = (long long)p.Hkv * ptot;
+  const long long C = plan_chunk(p, T);
+  const long long off = (long long)p.Hkv * pb + (long long)h * u;
+  if (u > 0 && r / p.G >= wb) {
     // Padding row of a shorter window: written as zeros by whichever kernel owns the
     // sequence (here if it was split; the attention kernel if it was whole).
-    const long long T0 = (long long)p.Hkv * p.pre_g[p.B];
-    const long long C0 = plan_chunk(p, T0);
-    const long long off0 = (long long)p.Hkv * p.pre_g[b] + (long long)h * u;
     int f0, l0;
-    plan_tile_ctas(p, off0, u, C0, &f0, &l0);
+    plan_tile_ctas(p, off, u, C, &f0, &l0);
     if (f0 != l0) reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
     return;
   }
@@ -46,9 +77,6 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
     if (lane == 0 && r == 0 && h == 0) atomicOr(&p.hdr->err, kErrSeqOverflow);
     return;
   }
-  const long long T = (long long)p.Hkv * p.pre_g[p.B];
-  const long long C = plan_chunk(p, T);
-  const long long off = (long long)p.Hkv * p.pre_g[b] + (long long)h * u;
   int c0, c1;
   plan_tile_ctas(p, off, u, C, &c0, &c1);
   if (c0 == c1) return;

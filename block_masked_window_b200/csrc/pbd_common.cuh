@@ -99,16 +99,21 @@ __host__ __device__ inline int window_of(const Problem& p, int b) {
 #endif
 }
 
-// Visible keys of sequence b, P_b + W_b (0 marks an invalid prefix or window length).
+// Visible keys P + w of a sequence with prefix P and window w (0 marks an invalid prefix or
+// window length).
+__host__ __device__ inline int visible_of(const Problem& p, int P, int w) {
+  if (P < 0 || w < 1 || w > p.W || (long long)P + w > (long long)p.S) return 0;
+  return P + w;
+}
+
+// Visible keys of sequence b, P_b + W_b.
 __host__ __device__ inline int visible_len(const Problem& p, int b) {
 #ifdef __CUDA_ARCH__
   int P = __ldg(p.seq_lens + b);
 #else
   int P = p.seq_lens[b];
 #endif
-  const int w = window_of(p, b);
-  if (P < 0 || w < 1 || w > p.W || (long long)P + w > (long long)p.S) return 0;
-  return P + w;
+  return visible_of(p, P, window_of(p, b));
 }
 
 // Key tiles of a sequence with n visible keys.
@@ -264,11 +269,15 @@ __host__ __device__ inline bool row_limits(const Problem& p) {
 }
 
 // Programmatic dependent launch. Every kernel of the library is launched so that it may start
-// while the previous kernel of the stream is still running; it signals right away that its own
-// successor may start too, and waits for its predecessor (completion and memory visibility)
-// before the first access to global memory. Every CTA executes the wait before it can exit,
-// so a kernel completes only after its predecessor did: the ordering is transitive along the
-// stream. Launched without the attribute, both instructions are no-ops.
+// while the previous kernel of the stream is still running, and waits for its predecessor
+// (completion and memory visibility) before the first access to global memory that a
+// predecessor may have written. Every CTA executes the wait before it can exit, so a kernel
+// completes only after its predecessor did: the ordering is transitive along the stream.
+// A kernel signals that its successor may start right away, except the attention kernels,
+// which signal after their wait: when the merge kernel starts, everything before the
+// attention kernel has completed, so the merge may read seq_lens and window_lens (which the
+// attention kernel does not write) before its own wait. Launched without the attribute, both
+// instructions are no-ops.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
