@@ -30,6 +30,14 @@
  * default stream) and return. They are reentrant. Run la_kv_append before la_pbd_attn on the
  * same stream (or use la_pbd_step, which does both).
  *
+ * Stream order: the kernels are launched with programmatic dependent launch, so each may
+ * start before the previous kernel of the stream has finished; each waits for it
+ * (griddepcontrol.wait) before reading anything a predecessor may have written, so stream
+ * order holds as usual. A caller's own kernel launched after one of these calls with
+ * programmatic dependent launch must, as that mechanism requires of any kernel, write
+ * nothing that the call reads (seq_lens, window_lens, the block table, q, the caches)
+ * before its own griddepcontrol.wait.
+ *
  * Errors: static arguments are checked on the host and reported synchronously (nothing is
  * enqueued on error). Per-sequence errors found on the device (seq_lens[b] < 0 or
  * seq_lens[b] + W > max_seq) never fault: that sequence's output rows are written as zeros,
