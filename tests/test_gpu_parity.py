@@ -118,6 +118,21 @@ def test_many_short_sequences(algo):
     assert_parity(gpu, ref, "300 short sequences")
 
 
+@pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
+@pytest.mark.parametrize("B", [31, 32, 33])
+def test_merge_plan_paths_at_32_sequences(B, algo):
+    """The merge derives a batch's plan itself for up to 32 sequences (one warp-wide scan of
+    seq_lens) and reads the prefix sums the attention kernel published for more: both sides
+    of that boundary, with whole and split sequences and one empty prefix."""
+    rng = np.random.default_rng(40 + B)
+    prefixes = tuple([0] + [int(x) for x in rng.integers(0, 2000, size=B - 1)])
+    wi = workloads.random_case(B, prefixes, 6, seed=40 + B)
+    li = wi.layers[0]
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, 6, algo=algo)
+    ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
+    assert_parity(gpu, ref, f"B={B}")
+
+
 def test_plan_fixed_cost_shapes():
     """34 sequences of 1-3 key tiles in a 1024-row cache: the tcgen05 plan charges each
     (sequence, KV head) two fixed-cost units, so with two units per CTA some CTAs hold only
