@@ -31,6 +31,11 @@ def test_reference_arm_prints_one_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert "layer calls of the tiny workload" in cb["sample"]
+    assert cb["cpu_model"]
+    # both threading configurations are timed; the faster one is the baseline
+    other = cb["other"]
+    assert other["value"] > 0 and other["value"] <= cb["value"] and other["unit"] == d["unit"]
+    assert 1 in (cb["cores"], other["cores"])
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
