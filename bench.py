@@ -1,16 +1,22 @@
 """Benchmark of the PBD window-attention path on B200.
 
 One step = one PBD decode step of the workload: for every layer, the window K/V append and
-the window attention (``la_pbd_step`` through the C ABI). Default workload: the single-image
-decode step (batch 1, 36 layers, prefix 1024 = 256 visual + 768 text/box tokens, window 6,
-16 query / 2 KV heads, d = 128, 1% of K channels x8), seed 1.
+the window attention (``la_pbd_step`` through the C ABI). Default workload: the long-context
+batch (8 sequences, prefix 32768, window 6, 16 query / 2 KV heads, d = 128, per-sequence K
+mean offset), seed 4, the largest of the target configurations; the other workloads are timed
+in the sweep, each with its own roofline block.
 
 Timing: inputs resident in HBM, several full copies of the workload rotated so that every step
 reads data that is not in L2 (working set > 2 x L2); the step is captured in a CUDA graph; W
 untimed warm-up steps; K timed steps between CUDA events on the launching stream with a
 barrier and synchronize on both sides; max over ranks. `e2e` repeats the measurement through
 the same C ABI with the step's inputs (Q, new K/V of every layer) copied from pinned host
-memory and the output copied back inside the timed region.
+memory and the output copied back inside the timed region (graph replays, copies on a second
+stream); `e2e_eager` does the same with the C-ABI calls made eagerly inside the timed region
+(no CUDA graph), as a caller without graphs would.
+
+`algo_compare` times the attention call of every workload with each attention kernel (tcgen05
+and CUDA cores) under the same protocol; the automatic kernel choice follows that table.
 
 Multi-GPU: replicas only (each rank runs its own independent batch; no collective on the data
 path; the timing uses one max-reduction).
@@ -190,23 +196,51 @@ def time_graphs(torch, graphs, steps, warmup, barrier):
     return start.elapsed_time(end)
 
 
-def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
+ALGO_NAMES = {1: "tcgen05", 2: "cuda_cores"}
+
+
+def supported_algos(wl):
+    """Attention kernels that take this workload: tcgen05 up to W * G = 80 query rows per KV
+    head, the CUDA-core kernel up to 128."""
+    R = wl.window * (wl.num_q_heads // wl.num_kv_heads)
+    return [a for a, lim in ((1, 80), (2, 128)) if R <= lim]
+
+
+def time_attention(args, bmw, torch, cfg_for, dev, seq, W, L, seq_of, ngraphs, inner, warmup,
+                   steps, barrier, max_over_ranks, device):
+    """Per-call time (us) of the attention call (attention + merge) of every layer, timed back
+    to back over the rotating copies, for the configuration `cfg_for`."""
+    ws = bmw.Workspace(cfg_for, W, device=device)
+    graphs = [capture(torch, lambda ds=seq_of(i): [run_attn_only(bmw, cfg_for, d, seq, W, ws, L) for d in ds])
+              for i in range(ngraphs)]
+    reps = max(1, math.ceil(max(steps, 20) / inner))
+    ms = max_over_ranks(time_graphs(torch, graphs, reps, warmup, barrier))
+    if bmw.la_pbd_check(ws) != 0:
+        raise RuntimeError("device-side status not OK after the attention timing")
+    del graphs
+    return ms * 1e3 / (reps * inner * L)
+
+
+def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks, e2e=True,
+            compare=True):
     wi = workloads.generate(wl)
     B, W = wl.batch, wl.window
     per_copy = (2 * wi.layers[0].k_cache.numel() * 2 + 3 * wi.layers[0].q.numel() * 2) * len(wi.layers)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     copies = max(2, min(args.max_copies, math.ceil(2.5 * l2 / max(per_copy, 1))))
     host, dev, seq, L = build_device_inputs(wi, copies, device)
-    cfg = bmw.Config.make(B, wl.num_q_heads, wl.num_kv_heads, wi.max_seq, algo=args.algo)
+    make_cfg = lambda algo: bmw.Config.make(B, wl.num_q_heads, wl.num_kv_heads, wi.max_seq,  # noqa: E731
+                                            algo=algo)
+    cfg = make_cfg(args.algo)
     R = W * (wl.num_q_heads // wl.num_kv_heads)
-    uses_tc = args.algo == 1 or (args.algo == 0 and R <= 64)
+    uses_tc = bmw.chosen_algo(cfg, W) == bmw.LA_ALGO_TCGEN05
     ws = bmw.Workspace(cfg, W, device=device)
 
     # One graph replay runs `inner` consecutive steps, each on the next copy in the rotation
     # (so every call still reads its inputs from HBM), so that workloads of a single layer
     # call are timed back to back like the 36 layer calls of a decode step, not one call per
     # graph launch.
-    inner = max(1, math.ceil(8 / L))
+    inner = max(d for d in range(1, max(1, math.ceil(8 / L)) + 1) if args.steps % d == 0)
     def seq_of(i):
         return [dev[(i * inner + j) % copies] for j in range(inner)]
     ngraphs = copies if inner == 1 else max(1, copies // math.gcd(copies, inner))
@@ -215,7 +249,7 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
     steps, warmup = args.steps, args.warmup
     clocks = ClockSampler(device.index if device.index is not None else 0)
     clocks.start()
-    replays = max(1, math.ceil(steps / inner))
+    replays = steps // inner   # exactly `steps` steps
     ms = time_graphs(torch, step_graphs, replays, warmup, barrier)
     clk = clocks.stop()
     ms = max_over_ranks(ms)
@@ -234,13 +268,16 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
     del floor_graph
 
     # Dominant kernel: the attention call of one layer (attention + split merge), timed alone
-    # over the same rotating copies.
-    attn_graphs = [capture(torch, lambda ds=seq_of(i): [run_attn_only(bmw, cfg, d, seq, W, ws, L) for d in ds])
-                   for i in range(ngraphs)]
-    reps = max(1, math.ceil(max(steps, 20) / inner))
-    ms_attn = time_graphs(torch, attn_graphs, reps, warmup, barrier)
-    ms_attn = max_over_ranks(ms_attn)
-    launch_us = ms_attn * 1e3 / (reps * inner * L)
+    # over the same rotating copies, with the kernel the step used; then every supported
+    # kernel, forced, for the comparison table.
+    launch_us = time_attention(args, bmw, torch, cfg, dev, seq, W, L, seq_of, ngraphs, inner,
+                               warmup, steps, barrier, max_over_ranks, device)
+    algo_us = {}
+    if compare:
+        for a in supported_algos(wl):
+            algo_us[ALGO_NAMES[a]] = time_attention(args, bmw, torch, make_cfg(a), dev, seq, W, L,
+                                                    seq_of, ngraphs, inner, warmup, steps, barrier,
+                                                    max_over_ranks, device)
     alg_bytes = workloads.algorithmic_bytes(wi.seq_lens.tolist(), W, wl.num_q_heads,
                                             wl.num_kv_heads, wl.head_dim)
     achieved = alg_bytes / (launch_us * 1e-6) / 1e9
@@ -249,8 +286,8 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
         raise RuntimeError("device-side status not OK after the benchmark")
 
     # End to end through the same API: inputs from pinned host memory, output back to host.
-    e2e = None
-    if not args.no_e2e:
+    e2e_res = e2e_eager = None
+    if e2e:
         # One step per replay here: each step copies its own inputs in and its output out.
         one_step = step_graphs if inner == 1 else [
             capture(torch, lambda d=d: run_step(bmw, cfg, d, seq, W, ws, L)) for d in dev]
@@ -277,12 +314,15 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
             in_ready[k].record(copy_s)
             used[k] = True
 
-        def run(n_steps):
+        def run(n_steps, graphed):
             upload(0)
             for i in range(n_steps):
                 k = i % copies
                 comp_s.wait_event(in_ready[k])
-                one_step[k].replay()
+                if graphed:
+                    one_step[k].replay()
+                else:
+                    run_step(bmw, cfg, dev[k], seq, W, ws, L)
                 done[k].record(comp_s)
                 if i + 1 < n_steps:
                     upload(i + 1)
@@ -291,30 +331,50 @@ def measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks):
                     h_out.copy_(dev[k]["out"], non_blocking=True)
             comp_s.wait_stream(copy_s)
 
-        run(warmup)
-        torch.cuda.synchronize()
-        barrier()
-        used = [False] * copies
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(comp_s)
-        run(steps)
-        e1.record(comp_s)
-        torch.cuda.synchronize()
-        barrier()
-        ms_e2e = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": aggregate_throughput(world, B, steps, ms_e2e), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ms_e2e / steps}
+        def timed(graphed):
+            nonlocal used
+            run(warmup, graphed)
+            torch.cuda.synchronize()
+            barrier()
+            used = [False] * copies
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(comp_s)
+            run(steps, graphed)
+            e1.record(comp_s)
+            torch.cuda.synchronize()
+            barrier()
+            ms_e = max_over_ranks(e0.elapsed_time(e1))
+            return {"value": aggregate_throughput(world, B, steps, ms_e), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": ms_e / steps}
+
+        e2e_res = timed(True)
+        e2e_res["how"] = "CUDA graph of the step's C-ABI calls per step; copies on a second stream"
+        e2e_eager = timed(False)
+        e2e_eager["how"] = "C-ABI calls made eagerly inside the timed region; copies on a second stream"
+        if bmw.la_pbd_check(ws) != 0:
+            raise RuntimeError("device-side status not OK after the end-to-end timing")
         del one_step
-    del step_graphs, attn_graphs
+    del step_graphs
     return {
         "wi": wi, "ms_per_step": ms_per_step, "value": value, "clocks": clk,
         "launch_us": launch_us, "alg_bytes": alg_bytes, "achieved_gbs": achieved,
-        "step_bytes": step_bytes, "copies": copies, "e2e": e2e, "layers": L,
+        "step_bytes": step_bytes, "copies": copies, "e2e": e2e_res, "e2e_eager": e2e_eager,
+        "layers": L, "algo_us": algo_us, "algo": ALGO_NAMES[bmw.chosen_algo(cfg, W)],
         # per layer: attention (with the append fused in on the tcgen05 path) + merge; the
         # CUDA-core path runs the append kernel too
         "launches_per_step": per_step_launches, "launch_floor": launch_floor,
     }
+
+
+def roofline_block(res, peak, peak_kind, name):
+    """Roofline of the dominant kernel (the attention call: attention + merge) of a workload."""
+    return {"bound": "hbm", "achieved": res["achieved_gbs"], "peak": peak, "unit": "GB/s",
+            "frac": res["achieved_gbs"] / peak, "peak_kind": peak_kind,
+            "frac_of_8tbs": res["achieved_gbs"] / 8000.0,
+            "traffic": stored_traffic(name),
+            "kernel": f"la_pbd_attn ({res['algo']} split-KV attention + merge), one layer",
+            "bytes_per_launch": res["alg_bytes"], "launch_us": res["launch_us"]}
 
 
 def measure_prefill(args, device, bmw, torch, barrier, max_over_ranks, T=16384, bs=6):
@@ -427,30 +487,37 @@ def cpu_baseline(wl, budget_s):
     return best
 
 
-def workload_label(wl):
+def workload_label(wl, world):
+    """The workload a line measures (identical in both arms' lines)."""
     return {"workload": wl.name, "batch": wl.batch, "layers": wl.layers,
             "prefix": wl.prefix if wl.prefix is not None else "ragged U{512..4096}+U{1..5}",
             "window": wl.window, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
-            "head_dim": wl.head_dim, "seed": wl.seed}
+            "head_dim": wl.head_dim, "seed": wl.seed, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (rotating copies of the whole workload)"}
+
+
+DEFAULT_SWEEP = "tiny,single_image,max_context,max_context_w1,ragged"
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="single_image", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="long", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--algo", type=int, default=0, help="0 auto, 1 tcgen05, 2 CUDA cores")
-    ap.add_argument("--sweep", default="max_context,max_context_w1,ragged,long",
+    ap.add_argument("--sweep", default=DEFAULT_SWEEP,
                     help="extra workloads measured for the prefix-length sweep ('' for none)")
     ap.add_argument("--max-copies", type=int, default=16)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-compare", action="store_true", help="skip the per-kernel timing table")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-prefill", action="store_true", help="skip the block-prefill line")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.steps = max(args.steps, 1)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -465,7 +532,7 @@ def main():
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1e3 * wl.batch / cb["value"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": workload_label(wl), "cpu_baseline": cb,
+                "config": workload_label(wl, args.gpus), "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
@@ -485,24 +552,27 @@ def main():
         torch.cuda.set_device(0)
     barrier, max_over_ranks = dist_helpers(world, device)
 
-    res = measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks)
+    compare = not args.no_compare
+    res = measure(args, rank, world, device, bmw, torch, wl, barrier, max_over_ranks,
+                  e2e=not args.no_e2e, compare=compare)
     peak, peak_kind = measured_peaks()
     sweep = []
-    for name in [s for s in args.sweep.split(",") if s]:
+    algo_compare = {wl.name: res["algo_us"]} if compare else {}
+    for name in [s for s in args.sweep.split(",") if s and s != wl.name]:
         swl = workloads.WORKLOADS[name]
         sargs = argparse.Namespace(**vars(args))
         sargs.steps = max(10, min(args.steps, 20))
-        sargs.no_e2e = True
-        r = measure(sargs, rank, world, device, bmw, torch, swl, barrier, max_over_ranks)
+        r = measure(sargs, rank, world, device, bmw, torch, swl, barrier, max_over_ranks,
+                    e2e=False, compare=compare)
+        if compare:
+            algo_compare[name] = r["algo_us"]
         sweep.append({
             "workload": name, "prefix": swl.prefix if swl.prefix is not None else "ragged",
             "batch": swl.batch, "window": swl.window, "layers": swl.layers,
             "window_steps_per_s": r["value"], "ms_per_step": r["ms_per_step"],
             "attn_launch_us": r["launch_us"], "attn_bytes_per_launch": r["alg_bytes"],
             "launch_floor_ms_per_step": r["launch_floor"]["ms_per_step"],
-            "achieved_gbs": r["achieved_gbs"], "frac_of_measured_hbm": r["achieved_gbs"] / peak,
-            "frac_of_8tbs": r["achieved_gbs"] / 8000.0,
-            "traffic": stored_traffic(name),
+            "roofline": roofline_block(r, peak, peak_kind, name), "clocks": r["clocks"],
         })
 
     prefill = None if args.no_prefill else measure_prefill(args, device, bmw, torch, barrier,
@@ -514,26 +584,23 @@ def main():
             dist.destroy_process_group()
         return
     cb = cpu_baseline(wl, args.cpu_budget) if (world == 1 and not args.no_cpu) else None
-    wi = res["wi"]
     line = {
         "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, per the workload recipe)",
-        "config": dict(workload_label(wl), **{
-            "parallelism": f"replicas x{world}", "l2": f"inputs > L2: {res['copies']} rotating copies",
-            "graph": "CUDA graph per step", "algo": args.algo}),
-        "roofline": {"bound": "hbm", "achieved": res["achieved_gbs"], "peak": peak,
-                     "unit": "GB/s", "frac": res["achieved_gbs"] / peak,
-                     "peak_kind": peak_kind, "traffic": stored_traffic(wl.name),
-                     "kernel": "la_pbd_attn (split-KV attention + merge), one layer",
-                     "bytes_per_launch": res["alg_bytes"], "launch_us": res["launch_us"]},
+        "config": workload_label(wl, world),
+        "run": {"graph": "CUDA graph per step", "algo": res["algo"], "algo_arg": args.algo,
+                "copies": res["copies"]},
+        "roofline": roofline_block(res, peak, peak_kind, wl.name),
         "gpu_launches": res["launches_per_step"] * args.steps,
-        "e2e": res["e2e"], "clocks": res["clocks"], "cpu_baseline": cb,
+        "e2e": res["e2e"], "e2e_eager": res["e2e_eager"], "clocks": res["clocks"],
+        "cpu_baseline": cb,
         "launch_floor": res["launch_floor"],
         "step_bytes": res["step_bytes"],
         "step_gbs": res["step_bytes"] / (res["ms_per_step"] * 1e-3) / 1e9,
         "sweep": sweep,
+        "algo_compare_us": algo_compare,
         "prefill": prefill,
     }
     print(json.dumps(line))

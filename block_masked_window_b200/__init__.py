@@ -17,7 +17,8 @@ __all__ = [
     "LaError", "Config", "load", "library_path", "la_version", "la_status_string",
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
     "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
-    "la_noop_chain", "la_pbd_attn_varwin",
+    "la_noop_chain", "la_pbd_attn_varwin", "la_pbd_algo", "chosen_algo",
+    "la_pbd_selftest_timeout",
     "la_pbd_step_varwin", "la_block_prefill", "la_pbd_attn_paged", "la_pbd_step_paged",
     "Workspace",
     "EXPORTED_SYMBOLS",
@@ -38,7 +39,7 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED",
 EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
                     "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
-                    "la_noop_chain",
+                    "la_noop_chain", "la_pbd_algo", "la_pbd_selftest_timeout",
                     "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill",
                     "la_pbd_attn_paged", "la_pbd_step_paged"]
 
@@ -119,6 +120,11 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_plan_params.argtypes = [i32, vp, vp]
     lib.la_noop_chain.restype = i32
     lib.la_noop_chain.argtypes = [i32, i32, i32, vp]
+    lib.la_pbd_algo.restype = i32
+    lib.la_pbd_algo.argtypes = [cfgp, i32]
+    lib.la_pbd_selftest_timeout.restype = i32
+    lib.la_pbd_selftest_timeout.argtypes = [cfgp, vp, vp, vp, vp, i32, vp, vp, sz, ctypes.c_int64,
+                                            vp]
     _LIB = lib
     return lib
 
@@ -285,6 +291,36 @@ def la_noop_chain(launches: int, ctas: int, threads: int, stream=None) -> None:
     """Enqueue `launches` empty kernels (launch-floor measurements)."""
     _check(load().la_noop_chain(int(launches), int(ctas), int(threads), _stream(stream)),
            "la_noop_chain")
+
+
+def la_pbd_selftest_timeout(cfg: Config, q, k_cache, v_cache, seq_lens, window_len: int, out,
+                            workspace: Workspace, wait_limit_ns: int, stream=None) -> None:
+    """Enqueue the failure-detection self-test (one attention call whose first S^T completion
+    is withheld, every wait limited to `wait_limit_ns`); la_pbd_check then gives 6
+    (LA_ERR_TIMEOUT)."""
+    W = int(window_len)
+    q_shape, cache_shape, _ = _shapes(cfg, W)
+    _check_tensor(q, "q", "bf16", q_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check_tensor(out, "out", "bf16", q_shape)
+    _check(load().la_pbd_selftest_timeout(ctypes.byref(cfg), _ptr(q), _ptr(k_cache),
+                                          _ptr(v_cache), _ptr(seq_lens), W, _ptr(out),
+                                          workspace.data_ptr(), workspace.nbytes,
+                                          int(wait_limit_ns), _stream(stream)),
+           "la_pbd_selftest_timeout")
+
+
+def la_pbd_algo(cfg: Config, window_len: int) -> int:
+    """The attention kernel (LA_ALGO_TCGEN05 or LA_ALGO_SIMT) the library runs for `cfg`."""
+    r = int(load().la_pbd_algo(ctypes.byref(cfg), int(window_len)))
+    if r < 0:
+        raise LaError(-r, "la_pbd_algo")
+    return r
+
+
+chosen_algo = la_pbd_algo
 
 
 def la_pbd_plan_params(algo: int):

@@ -12,7 +12,8 @@
 // adds its fp32 p values to NQ partial sums kept in its own TMEM lane, after it has handed
 // the tile's P^T to the MMA, and the 128 lanes are reduced once per segment. So the single
 // MMA-issuing thread issues 16 instructions per tile, not 24.
-// NQ = R rounded up to 16 (48 for the PBD window of 6 rows x 8 grouped heads). P is split
+// NQ = R rounded up to 16 (48 for the PBD window of 6 rows x 8 grouped heads; up to 80, the
+// window of 10 rows that the RKLLM engine sends after 5 accepted tokens). P is split
 // into P_hi + P_lo (both bf16, residual ~2^-17 P) so that the bf16 tensor-core product keeps
 // fp32-level accuracy; both halves ride in one N = 2 NQ MMA that reads the V tile once.
 //
@@ -44,9 +45,11 @@
 // memory for one TMA store; a split sequence's fp32 partial rows go straight from registers
 // to their slot.
 //
-// Every mbarrier wait is bounded: after ~2 s the CTA raises the sticky timeout flag in the
-// workspace header, the other roles stop at their next wait, in-flight copies and MMAs are
-// drained with bounded waits, TMEM is freed and the kernel returns.
+// Every mbarrier wait is bounded: after a limit (2 s by default, set per call) the CTA raises
+// the sticky timeout flag in the workspace header, the other roles stop at their next wait,
+// in-flight copies and MMAs are drained with bounded waits, TMEM is freed and the kernel
+// returns. A self-test option withholds the first S^T completion signal so that this path
+// runs (la_pbd_selftest_timeout).
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 #include "tc_util.cuh"
@@ -60,7 +63,7 @@ using namespace tc;
 constexpr int kNT = kTileKeys;          // 128 keys per tile
 constexpr int kSegUnits = 2;            // plan units charged per segment (tc_segment_units)
 constexpr int kKStages = 2;
-constexpr int kSBufs = 4;               // S^T buffers in TMEM: QK may run kSBufs-1 tiles ahead
+constexpr int kSBufs = 4;               // S^T buffers in TMEM (most): QK may run kSBufs-1 tiles ahead
 constexpr int kThreadsTc = 224;
 constexpr int kTmemCols = 512;
 constexpr int kHalfBytes = kNT * 128;   // 128 rows x 128 B: one swizzle column of a K/V tile
@@ -89,6 +92,15 @@ constexpr int kBarKRaw = kBarDrain + 1;              // [kKStages]: K tiles of a
 constexpr int kBarVRaw = kBarKRaw + kKStages;         // [kMaxVStages]: V tiles of a fused append
 constexpr int kNumBars = kBarVRaw + kMaxVStages;
 
+// Buffers of the rows' operands for a given NQ: up to 64 rows, four S^T buffers in TMEM and
+// a double-buffered P^T in shared memory (the softmax of tile t + 1 writes P^T while the PV
+// product of tile t reads the other buffer); at 80 rows TMEM holds three S^T buffers
+// ((3 + 3) x 80 of its 512 columns) and P^T is single-buffered, so that the K and V rings still
+// fit in shared memory (the softmax of tile t + 1 computes its probabilities first and waits
+// for the PV product of tile t only before storing them).
+__host__ __device__ constexpr int tc_sbufs(int nq) { return nq <= 64 ? kSBufs : 3; }
+__host__ __device__ constexpr int tc_pbufs(int nq) { return nq <= 64 ? 2 : 1; }
+
 // Shared-memory plan for a given NQ and V ring depth.
 struct TcLayout {
   int k, v, q, p, bar, misc, vote, wmax, lim, mref, alpha, pre, end;
@@ -102,7 +114,7 @@ __host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, in
   L.v = L.k + kKStages * kTileBytes;
   L.q = L.v + vstages * kTileBytes;
   L.p = L.q + qbufs * 2 * nq * 128;         // Q: qbufs buffers x two 64-channel halves
-  L.bar = L.p + 2 * nq * 512;               // P^T: 2 buffers x 2*nq/8 row groups of 2048 B
+  L.bar = L.p + tc_pbufs(nq) * nq * 512;    // P^T: buffers of 2*nq/8 row groups of 2048 B
   L.misc = a16(L.bar + kNumBars * 8);       // tmem slot, abort flag
   L.vote = L.misc + 16;                     // (unused slot kept for alignment)
   L.wmax = L.vote + 32;                     // [2][4][nq] floats
@@ -258,12 +270,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     pbd_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                        const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
                        Problem p, int ring) {
-  static_assert(NQ % 16 == 0 && NQ >= 16 && NQ <= 64, "NQ");
+  static_assert(NQ % 16 == 0 && NQ >= 16 && NQ <= 80, "NQ");
   constexpr int kQHalf = NQ * 128;                 // bytes of one 64-channel half of Q
-  constexpr int kColS = 0;                         // S^T buffers at [0, kSBufs NQ)
-  constexpr int kColO = kSBufs * NQ;               // O^T (hi | lo)
-  constexpr int kColL = (kSBufs + 2) * NQ;         // row-sum partials of each key lane
-  static_assert((kSBufs + 3) * NQ <= kTmemCols, "TMEM columns");
+  constexpr int kSB = tc_sbufs(NQ);                // S^T buffers
+  constexpr int kPB = tc_pbufs(NQ);                // P^T buffers
+  constexpr int kColS = 0;                         // S^T buffers at [0, kSB NQ)
+  constexpr int kColO = kSB * NQ;                  // O^T (hi | lo)
+  constexpr int kColL = (kSB + 2) * NQ;            // row-sum partials of each key lane
+  static_assert((kSB + 3) * NQ <= kTmemCols, "TMEM columns");
+  static_assert(kSB <= kSBufs, "S barriers");
   constexpr uint32_t kIdescQK = idesc_f16(128, NQ, 0, 0);
   constexpr uint32_t kIdescPV = idesc_f16(128, 2 * NQ, 1, 1);
 
@@ -282,7 +297,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   int* warp_tot = pre + round_up(p.B + 1, 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  Ctl ctl{abort_flag, p.hdr};
+  Ctl ctl{abort_flag, p.hdr, p.wait_limit_ns};
   if (tid == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
@@ -514,7 +529,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       uint32_t sQseg = sQ;   // Q buffer of the current segment
       auto issue_qk = [&](int gg) {
         const uint32_t kb = sK + (gg % kKStages) * kTileBytes;
-        const uint32_t d = tmem + kColS + (uint32_t)((gg % kSBufs) * NQ);
+        const uint32_t d = tmem + kColS + (uint32_t)((gg % kSB) * NQ);
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
           const uint32_t ka = kb + (kk >> 2) * kHalfBytes + (kk & 3) * 32;
@@ -526,7 +541,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const uint32_t vb = sV + (gg % vstages) * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kNT / 16; ++kk) {
-          const uint64_t pdesc = sdesc(sP + (gg & 1) * (NQ * 512) + kk * 256, 128, 2048, 0);
+          const uint64_t pdesc = sdesc(sP + (gg % kPB) * (NQ * 512) + kk * 256, 128, 2048, 0);
           const uint32_t acc = (first && kk == 0) ? 0u : 1u;
           umma(tmem + kColO, sdesc(vb + kk * 2048, kHalfBytes, 1024, 2), pdesc, kIdescPV, acc);
         }
@@ -537,7 +552,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (!mbar_wait(bar(kBarQFull + qs), (nseg / qbufs) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         sQseg = sQ + qs * 2 * kQHalf;
-        // Issue S^T(t) as soon as K(t) has landed and its S buffer is free (P(t-2) consumed),
+        // Issue S^T(t) as soon as K(t) has landed and its S buffer is free (P(t-kSB+1) consumed),
         // and O^T += V^T P^T(t) as soon as P(t) and V(t) are ready, whichever comes first.
         const int g0 = g;
         int nqk = 0, npv = 0;
@@ -545,13 +560,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         uint32_t spins = 0;
         while (npv < nt) {
           bool prog = false;
-          const bool want_qk = nqk < nt && nqk <= npv + kSBufs - 1;
+          const bool want_qk = nqk < nt && nqk <= npv + kSB - 1;
           const bool want_pv = npv < nqk;
           if (want_qk != want_pv) {
             // One event pending: a (bounded) blocking wait is cheaper than polling.
             const bool got = want_qk
                 ? mbar_wait(bar(kBarKFull + (g0 + nqk) % kKStages), ((g0 + nqk) / kKStages) & 1, ctl)
-                : (mbar_wait(bar(kBarPFull + ((g0 + npv) & 1)), ((g0 + npv) >> 1) & 1, ctl) &&
+                : (mbar_wait(bar(kBarPFull + (g0 + npv) % kPB), ((g0 + npv) / kPB) & 1, ctl) &&
                    mbar_wait(bar(kBarVFull + (g0 + npv) % vstages), ((g0 + npv) / vstages) & 1, ctl));
             if (!got) { ok = false; break; }
           }
@@ -560,7 +575,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             if (mbar_test(bar(kBarKFull + gq % kKStages), (gq / kKStages) & 1)) {
               tc_fence_after();
               issue_qk(gq);
-              umma_commit(bar(kBarSFull + gq % kSBufs));
+              // (Self-test of the failure detection: the first completion is withheld, so the
+              // softmax warps' bounded wait for it runs out.)
+              if (!(p.stall_test && gq == 0)) umma_commit(bar(kBarSFull + gq % kSB));
               umma_commit(bar(kBarKEmpty + gq % kKStages));
               if (nqk == nt - 1) umma_commit(bar(kBarQEmpty + qs));
               ++nqk;
@@ -569,11 +586,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
           if (want_pv) {
             const int gp = g0 + npv;
-            if (mbar_test(bar(kBarPFull + (gp & 1)), (gp >> 1) & 1) &&
+            if (mbar_test(bar(kBarPFull + gp % kPB), (gp / kPB) & 1) &&
                 mbar_test(bar(kBarVFull + gp % vstages), (gp / vstages) & 1)) {
               tc_fence_after();
               issue_pv(gp, npv == 0);
-              umma_commit(bar(kBarOFull + (gp & 1)));
+              umma_commit(bar(kBarOFull + gp % kPB));
               umma_commit(bar(kBarVEmpty + gp % vstages));
               ++npv;
               prog = true;
@@ -589,7 +606,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           __nanosleep(32);
           if ((++spins & 63u) == 0) {
             if (*abort_flag) { ok = false; break; }
-            if (now_ns() - t_prog > kWaitLimitNs) {
+            if (now_ns() - t_prog > p.wait_limit_ns) {
               *abort_flag = 1;
               atomicOr(&p.hdr->err, kErrTimeout);
               ok = false;
@@ -636,11 +653,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const int jt = sg.j0 + t * kNT;
         const int key = jt + row;
         const bool key_ok = key < sg.j1;
-        const uint32_t s_addr = lane_addr + kColS + (gt % kSBufs) * NQ;
-        if (!mbar_wait(bar(kBarSFull + gt % kSBufs), (gt / kSBufs) & 1, ctl)) { ok = false; break; }
+        const uint32_t s_addr = lane_addr + kColS + (gt % kSB) * NQ;
+        if (!mbar_wait(bar(kBarSFull + gt % kSB), (gt / kSB) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         // P^T is written as hi/lo row groups, one 16-byte store per 8 rows.
-        const uint32_t prow = sP + (gt & 1) * (NQ * 512) + (uint32_t)((row >> 3) * 128 + (row & 7) * 16);
+        const uint32_t prow = sP + (gt % kPB) * (NQ * 512) + (uint32_t)((row >> 3) * 128 + (row & 7) * 16);
         // A segment's first tile has no references yet: it always takes the exact-maximum
         // path below.
         bool rescale = true;
@@ -674,9 +691,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           rescale = softmax_bar_or(exceeds);
           if (!rescale) {
             hot = true;
-            // The product that read this P^T buffer two tiles ago must be done.
-            if (gt > 1) {
-              if (!mbar_wait(bar(kBarOFull + (gt & 1)), ((gt - 2) >> 1) & 1, ctl)) { ok = false; break; }
+            // The product that last read this P^T buffer (tile gt - kPB) must be done.
+            if (gt >= kPB) {
+              const int gr = gt - kPB;
+              if (!mbar_wait(bar(kBarOFull + gr % kPB), (gr / kPB) & 1, ctl)) { ok = false; break; }
               tc_fence_after();
             }
 #pragma unroll
@@ -717,9 +735,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             alpha_s[q] = (mn == -INFINITY) ? 1.f : fast_exp2(mo - mn);
           }
           // The previous PV product (and so every earlier one) must be complete before O and l
-          // are rescaled in place.
+          // are rescaled in place (and before a single P^T buffer is rewritten).
           if (gt > 0) {
-            if (!mbar_wait(bar(kBarOFull + ((gt - 1) & 1)), ((gt - 1) >> 1) & 1, ctl)) { ok = false; break; }
+            if (!mbar_wait(bar(kBarOFull + (gt - 1) % kPB), ((gt - 1) / kPB) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
           }
           softmax_bar();
@@ -792,7 +810,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(kBarPFull + (gt & 1)));
+        mbar_arrive(bar(kBarPFull + gt % kPB));
         if (hot) {
           // Off the MMA's critical path: this tile's p joins the row-sum partials of this
           // key lane (the previous tile's partial stores have completed: every tile ends
@@ -812,7 +830,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (!ok) break;
       const int glast = g + nt - 1;
       g += nt;
-      if (!mbar_wait(bar(kBarOFull + (glast & 1)), (glast >> 1) & 1, ctl)) { ok = false; break; }
+      if (!mbar_wait(bar(kBarOFull + glast % kPB), (glast / kPB) & 1, ctl)) { ok = false; break; }
       tc_fence_after();
 
       // Epilogue: O^T row `row` (one channel) of a whole sequence is normalised, staged in the
@@ -944,7 +962,7 @@ static int tc_nq(int R) { return round_up(R, 16); }
 // on a ragged batch of 64 sequences when it costs a V stage).
 static int tc_ring(int nq, int B) {
   const int limit = 227 * 1024 - 1024;
-  const int options[5][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}, {1, 1}};
+  const int options[5][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}, {1, 1}};   // {V stages, Q buffers}
   for (auto& o : options)
     if (tc_layout(nq, o[0], o[1], B).end <= limit) return o[0] | (o[1] << 8);
   return 0;
@@ -990,6 +1008,7 @@ cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tma
     LA_TC_CASE(32)
     LA_TC_CASE(48)
     LA_TC_CASE(64)
+    LA_TC_CASE(80)
     default: return cudaErrorInvalidValue;
   }
 #undef LA_TC_CASE

@@ -57,14 +57,14 @@ la_status check_cfg(const la_pbd_cfg* cfg, int32_t W) {
   if ((long long)cfg->batch * cfg->num_kv_heads > 65535) return LA_ERR_UNSUPPORTED;
   const long long R = (long long)W * (cfg->num_q_heads / cfg->num_kv_heads);
   if (R > 128) return LA_ERR_UNSUPPORTED;
-  if (cfg->algo == LA_ALGO_TCGEN05 && R > 64) return LA_ERR_UNSUPPORTED;
+  if (cfg->algo == LA_ALGO_TCGEN05 && R > 80) return LA_ERR_UNSUPPORTED;
   return LA_OK;
 }
 
 // Kernel choice for a validated configuration.
 int pick_algo(const la_pbd_cfg* cfg, int R) {
   if (cfg->algo != LA_ALGO_AUTO) return cfg->algo;
-  return (R <= 64) ? LA_ALGO_TCGEN05 : LA_ALGO_SIMT;
+  return (R <= 80) ? LA_ALGO_TCGEN05 : LA_ALGO_SIMT;
 }
 
 size_t slots_for(const la_pbd_cfg* cfg, int sms) {
@@ -83,6 +83,7 @@ la_status fill_problem(const la_pbd_cfg* cfg, int32_t W, Problem* p) {
   p->rows_pad = la::round_up(p->R, 16);
   p->mask_mode = cfg->mask_mode;
   p->scale_log2 = cfg->scale * 1.4426950408889634f;
+  p->wait_limit_ns = la::kDefaultWaitLimitNs;
   return LA_OK;
 }
 
@@ -112,6 +113,12 @@ const char* la_status_string(la_status s) {
     case LA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
   }
   return "unknown status";
+}
+
+int32_t la_pbd_algo(const la_pbd_cfg* cfg, int32_t W) {
+  const la_status st = check_cfg(cfg, W);
+  if (st != LA_OK) return -(int32_t)st;
+  return pick_algo(cfg, W * (cfg->num_q_heads / cfg->num_kv_heads));
 }
 
 size_t la_pbd_workspace_bytes(const la_pbd_cfg* cfg, int32_t W) {
@@ -172,13 +179,21 @@ struct Paging {
   int pages_per_seq = 0, page_size = 0, num_pages = 0;
 };
 
+// Self-test of the device-side failure detection (la_pbd_selftest_timeout).
+struct Selftest {
+  long long wait_limit_ns = la::kDefaultWaitLimitNs;
+  int stall = 0;
+};
+
 la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* seq_lens,
                       const int32_t* window_lens, int32_t W, void* out, void* workspace,
                       const void* k_new, const void* v_new, void* stream,
-                      const Paging& pg = Paging()) {
+                      const Paging& pg = Paging(), const Selftest& st = Selftest()) {
   Problem p;
   fill_problem(cfg, W, &p);
+  p.wait_limit_ns = st.wait_limit_ns;
+  p.stall_test = st.stall;
   p.window_lens = window_lens;
   if (pg.block_table) {
     p.block_table = pg.block_table;
@@ -392,6 +407,7 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
   p.T = t_max;
   p.bs = block_size;
   p.scale_log2 = cfg->scale * 1.4426950408889634f;
+  p.wait_limit_ns = la::kDefaultWaitLimitNs;
   CUtensorMap mq, mk, mv;
   if (la::make_prefill_maps(p, &mq, &mk, &mv) != cudaSuccess) return LA_ERR_CUDA;
   cudaError_t e = la::launch_prefill_tc(p, &mq, &mk, &mv, (cudaStream_t)stream);
@@ -449,6 +465,23 @@ la_status la_pbd_step_paged(const la_pbd_cfg* cfg, const void* q, const void* k_
   pg.num_pages = num_pages;
   return attn_launch(cfg, q, k_pool, v_pool, seq_lens, nullptr, W, out, workspace, k_new,
                      v_new, stream, pg);
+}
+
+la_status la_pbd_selftest_timeout(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* seq_lens, int32_t W,
+                                   void* out, void* workspace, size_t workspace_bytes,
+                                   int64_t wait_limit_ns, void* stream) {
+  if (wait_limit_ns < 1000 || wait_limit_ns > la::kDefaultWaitLimitNs) return LA_ERR_INVALID_ARG;
+  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  if (pick_algo(cfg, W * (cfg->num_q_heads / cfg->num_kv_heads)) != LA_ALGO_TCGEN05)
+    return LA_ERR_UNSUPPORTED;
+  Selftest t;
+  t.wait_limit_ns = wait_limit_ns;
+  t.stall = 1;
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, nullptr, W, out, workspace, nullptr,
+                     nullptr, stream, Paging(), t);
 }
 
 la_status la_pbd_check(void* workspace, void* stream) {

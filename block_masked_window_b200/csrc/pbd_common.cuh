@@ -22,6 +22,7 @@ constexpr int kHeadDim = 128;
 constexpr int kMaxBatch = 4096;
 constexpr int kMaxWindow = 16;
 constexpr int kHeaderBytes = 256;
+constexpr long long kDefaultWaitLimitNs = 2000000000LL;   // bounded device-side waits: ~2 s
 
 // Sticky error bits in the workspace header (first 32-bit word).
 constexpr uint32_t kErrSeqOverflow = 1u;
@@ -63,6 +64,8 @@ struct Problem {
   int c_min;                    // minimum units per CTA
   int seg_units;                // plan units charged per (sequence, KV head) besides its tiles
   float scale_log2;             // scale * log2(e)
+  long long wait_limit_ns;      // limit of every bounded device-side wait (tcgen05 kernel)
+  int stall_test;               // self-test: the first S^T completion is never signalled
 };
 
 // Launch parameters of the block-causal prefill kernel.
@@ -76,6 +79,7 @@ struct PrefillProblem {
   int B, Hq, Hkv, G, S, T;      // T = padded token count of q / out
   int bs;                       // block size of the block mask
   float scale_log2;
+  long long wait_limit_ns;      // limit of every bounded device-side wait
 };
 
 __host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }

@@ -39,7 +39,7 @@ size_t simt_smem_bytes(int R, int B);
 cudaError_t simt_max_ctas_per_sm(int R, int B, int* ctas);
 cudaError_t launch_attn_simt(const Problem& p, cudaStream_t stream);
 
-// tcgen05 + TMA split-KV attention (R <= 64).
+// tcgen05 + TMA split-KV attention (R <= 80).
 size_t tc_smem_bytes(int R, int B);
 cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tmap_v,
                            const void* tmap_q, const void* tmap_o, cudaStream_t stream);

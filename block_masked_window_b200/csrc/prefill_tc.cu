@@ -16,11 +16,17 @@
 // softmax threads own query row r (TMEM lane r), one per key half: each reads its 64 scores
 // from TMEM, keeps its lazy reference maximum (raised only when a score exceeds it by 2^8;
 // the warp then rescales its O_h rows after the previous PV product has completed) and row
-// sum in registers, and writes its half of the row of P (bf16) into shared memory in the
-// 128-byte-swizzled K-major layout the MMA reads. With no exchange between the halves per
-// tile, the two warps sharing a scheduler drift apart, so one's exponentials overlap the
-// other's maxima and TMEM reads. At the end the pair merges (m, l, O_0, O_1) and each thread
-// normalises and stores 64 of the row's 128 output channels.
+// sum in registers, and writes its half of the row of P into shared memory in the
+// 128-byte-swizzled K-major layout the MMA reads. P is written as two bf16 parts, P = P_hi +
+// P_lo (P_lo = bf16(P - P_hi), residual ~2^-17 P), and each PV product is issued for both
+// parts, so the product keeps fp32-level accuracy in P: a single bf16 rounding of P would add
+// a relative L2 error of ~1e-3 to the output, on top of the ~1.7e-3 of its own bf16 rounding.
+// The P region of a key half is single-buffered: the softmax of tile t computes its
+// probabilities first and waits for the PV product of tile t - 1 only before storing them.
+// With no exchange between the halves per tile, the two warps sharing a scheduler drift
+// apart, so one's exponentials overlap the other's maxima and TMEM reads. At the end the pair
+// merges (m, l, O_0, O_1) and each thread normalises and stores 64 of the row's 128 output
+// channels.
 //
 // Roles (352 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 10 TMA for the V
 // ring, warp 1 TMEM owner and MMA issuer, warps 2..9 softmax (warps w and w + 4 share the TMEM
@@ -43,6 +49,7 @@ constexpr int kPfThreads = 352;         // 11 warps
 constexpr int kPfStages = 2;             // K and V ring depth
 constexpr int kPHalf = 128 * 128;        // one 64-column half of a 128-row bf16 tile (16 KB)
 constexpr int kPTile = 2 * kPHalf;       // 32 KB
+constexpr int kPRegion = 2 * kPHalf;     // P of one key half: P_hi (16 KB) then P_lo (16 KB)
 constexpr float kPfLazy = 8.f;           // log2 units
 constexpr int kPfTmemCols = 512;
 constexpr int kColS = 0;                 // S: 2 buffers x 128 columns
@@ -54,17 +61,17 @@ constexpr int kBKEmpty = kBKFull + kPfStages;     // [kPfStages]
 constexpr int kBVFull = kBKEmpty + kPfStages;     // [kPfStages]
 constexpr int kBVEmpty = kBVFull + kPfStages;     // [kPfStages]
 constexpr int kBSFull = kBVEmpty + kPfStages;     // [2]
-constexpr int kBPFull = kBSFull + 2;              // [key half][P buffer], 128 arrivals each
-constexpr int kBOFull = kBPFull + 4;              // [key half][P buffer]
+constexpr int kBPFull = kBSFull + 2;              // [key half][tile parity], 128 arrivals each
+constexpr int kBOFull = kBPFull + 4;              // [key half][tile parity]
 constexpr int kBDrain = kBOFull + 4;
 constexpr int kBNum = kBDrain + 1;
 
-// Shared memory: Q | K ring | V ring | P x 2 | barriers | misc.
+// Shared memory: Q | K ring | V ring | P (two key halves x {P_hi, P_lo}) | barriers | misc.
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kPTile;
 constexpr int kOffV = kOffK + kPfStages * kPTile;
 constexpr int kOffP = kOffV + kPfStages * kPTile;
-constexpr int kOffBar = kOffP + 2 * kPTile;
+constexpr int kOffBar = kOffP + 2 * kPRegion;
 constexpr int kOffMisc = kOffBar + kBNum * 8;
 constexpr int kPfSmem = kOffMisc + 16;
 // The final (m, l) exchange of the two halves ([2][2 halves][128 rows] floats) reuses the Q
@@ -75,11 +82,24 @@ constexpr size_t kPfSmemAlloc = (size_t)kPfSmem + 1024;   // + alignment slack
 // Named barrier 1 over the 256 softmax threads.
 __device__ __forceinline__ void pf_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-// 8 bf16 probabilities (keys 8 k8 .. 8 k8 + 7) of row r into the swizzled K-major P tile.
-__device__ __forceinline__ void store_p16(uint32_t prow, int k8, int r, const uint32_t (&pk)[4]) {
-  const uint32_t a = prow + (uint32_t)((k8 >> 3) * kPHalf + (((k8 & 7) ^ (r & 7)) << 4));
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[0]), "r"(pk[1]),
-               "r"(pk[2]), "r"(pk[3]));
+// 8 probabilities (keys 8 k8 .. 8 k8 + 7 of a key half) of row r as bf16 P_hi and P_lo into
+// the swizzled K-major P region of that half; `prow` is row r of its P_hi part.
+__device__ __forceinline__ void store_p_hilo(uint32_t prow, int k8, int r, const float* x) {
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float a = x[2 * e], b = x[2 * e + 1];
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+    hi[e] = *reinterpret_cast<uint32_t*>(&h2);
+    const float ha = __uint_as_float(hi[e] << 16), hb = __uint_as_float(hi[e] & 0xFFFF0000u);
+    __nv_bfloat162 l2 = __floats2bfloat162_rn(a - ha, b - hb);
+    lo[e] = *reinterpret_cast<uint32_t*>(&l2);
+  }
+  const uint32_t a = prow + (uint32_t)(((k8 ^ (r & 7)) << 4));
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(hi[0]), "r"(hi[1]),
+               "r"(hi[2]), "r"(hi[3]));
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a + kPHalf), "r"(lo[0]),
+               "r"(lo[1]), "r"(lo[2]), "r"(lo[3]));
 }
 
 }  // namespace
@@ -101,7 +121,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.G;
   const int i0 = tile * kBM;
-  Ctl ctl{abort_flag, p.hdr};
+  Ctl ctl{abort_flag, p.hdr, p.wait_limit_ns};
 
   pdl_trigger();
   if (tid == 0) {
@@ -218,7 +238,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             prog = true;
           }
         }
-        // O_h += P_h(t) V_h(t): P columns (keys) [64h, 64h + 64) times V rows [64h, 64h + 64).
+        // O_h += (P_hi + P_lo)_h(t) V_h(t): P columns (keys) [64h, 64h + 64) times V rows
+        // [64h, 64h + 64), once for each bf16 part of P.
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int t = npv[hh];
@@ -227,12 +248,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (mbar_test(bar(kBPFull + 2 * hh + (t & 1)), (t >> 1) & 1) &&
                 mbar_test(bar(kBVFull + s), (t / kPfStages) & 1)) {
               tc_fence_after();
-              const uint32_t pb = sP + (t & 1) * kPTile + hh * kPHalf;
+              const uint32_t pb = sP + hh * kPRegion;
               const uint32_t vb = sV + s * kPTile + hh * 4 * 2048;
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                umma(tmem + kColO + hh * 128, sdesc(pb + kk * 32, 16, 1024, 2),
-                     sdesc(vb + kk * 2048, kPHalf, 1024, 2), kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t vd = sdesc(vb + kk * 2048, kPHalf, 1024, 2);
+                umma(tmem + kColO + hh * 128, sdesc(pb + kk * 32, 16, 1024, 2), vd, kIdO,
+                     (t > 0 || kk > 0) ? 1u : 0u);
+                umma(tmem + kColO + hh * 128, sdesc(pb + kPHalf + kk * 32, 16, 1024, 2), vd, kIdO, 1u);
+              }
               umma_commit(bar(kBOFull + 2 * hh + (t & 1)));
               ++npv[hh];
               // The V tile is free once both halves' products of it are issued.
@@ -249,7 +273,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         __nanosleep(32);
         if ((++spins & 63u) == 0) {
           if (*abort_flag) { ok = false; break; }
-          if (now_ns() - t_prog > kWaitLimitNs) {
+          if (now_ns() - t_prog > p.wait_limit_ns) {
             *abort_flag = 1;
             atomicOr(&p.hdr->err, kErrTimeout);
             ok = false;
@@ -324,30 +348,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         tc_wait_st();
       }
-      // This half of the P buffer was last read by this half's PV product two tiles ago.
-      if (t > 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + 2 * half + (t & 1)), ((t - 2) >> 1) & 1, ctl))) { ok = false; break; }
-        tc_fence_after();
-      }
-      // p = 2^(x c2 - m_ref), bf16 into this half of the swizzled K-major P row, 8 keys per
-      // 16-byte store. (Masked scores are -inf: ex2.approx gives exactly 0 for them.)
-      const uint32_t prow = sP + (t & 1) * kPTile + (uint32_t)r * 128u;
+      // p = 2^(x c2 - m_ref) in fp32 (masked scores are -inf: ex2.approx gives exactly 0 for
+      // them), and this tile's part of the row sum.
       const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k8 = 0; k8 < 8; ++k8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const float a = fast_exp2(fmaf(x[8 * k8 + e], c2, -mref));
-          const float bq = fast_exp2(fmaf(x[8 * k8 + e + 1], c2, -mref));
-          ls[e >> 1] += a + bq;
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bq);
-          pk[e >> 1] = *reinterpret_cast<uint32_t*>(&v2);
-        }
-        store_p16(prow, 8 * half + k8, r, pk);
+      for (int e = 0; e < 64; ++e) {
+        x[e] = fast_exp2(fmaf(x[e], c2, -mref));
+        ls[e & 3] += x[e];
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // This half's P region was last read by this half's PV product of the previous tile.
+      if (t > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + 2 * half + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl))) { ok = false; break; }
+        tc_fence_after();
+      }
+      // P_hi and P_lo into this half's swizzled K-major P rows, 8 keys per 16-byte store each.
+      const uint32_t prow = sP + half * kPRegion + (uint32_t)r * 128u;
+#pragma unroll
+      for (int k8 = 0; k8 < 8; ++k8) store_p_hilo(prow, k8, r, x + 8 * k8);
       // Keys of this half past the visible range (last tile): zero their V rows so that
       // 0 * x cannot become NaN in the product (those rows may hold anything).
       const int valid = min(kBN, kmax - t * kBN);

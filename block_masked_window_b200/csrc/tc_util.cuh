@@ -12,8 +12,6 @@
 namespace la {
 namespace tc {
 
-constexpr long long kWaitLimitNs = 2000000000LL;   // bounded waits: ~2 s, then abort
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -75,6 +73,7 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 struct Ctl {
   volatile int* abort_flag;
   WsHeader* hdr;
+  long long limit_ns;    // a wait gives up (and the CTA aborts) after this long
 };
 
 // Bounded wait for the completion of phase `parity`. Returns false when the CTA is aborting.
@@ -85,7 +84,7 @@ static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, con
     if (mbar_try(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*ctl.abort_flag) return false;
-      if (now_ns() - t0 > kWaitLimitNs) {
+      if (now_ns() - t0 > ctl.limit_ns) {
         *ctl.abort_flag = 1;
         atomicOr(&ctl.hdr->err, kErrTimeout);
         return false;

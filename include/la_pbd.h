@@ -74,7 +74,7 @@ enum {
 /* Kernel selection. */
 enum {
   LA_ALGO_AUTO = 0,      /* tensor-core kernel when supported, else CUDA cores             */
-  LA_ALGO_TCGEN05 = 1,   /* tcgen05 (TMEM accumulators) + TMA staging; W * Hq/Hkv <= 64    */
+  LA_ALGO_TCGEN05 = 1,   /* tcgen05 (TMEM accumulators) + TMA staging; W * Hq/Hkv <= 80    */
   LA_ALGO_SIMT = 2       /* fp32 CUDA-core kernel; W * Hq/Hkv <= 128                       */
 };
 
@@ -94,6 +94,15 @@ int32_t la_version(void);
 
 /* Static text for a status code (never NULL). */
 const char* la_status_string(la_status status);
+
+/*
+ * The attention kernel that la_pbd_attn / la_pbd_step / la_pbd_attn_varwin would run for this
+ * configuration and (longest) window length: LA_ALGO_TCGEN05 or LA_ALGO_SIMT. With
+ * cfg->algo = LA_ALGO_AUTO the choice follows the measured per-workload timing of both kernels
+ * on B200 (the tensor-core kernel wherever it supports the shape, W * Hq/Hkv <= 80). Host
+ * only; returns -la_status for an invalid or unsupported configuration.
+ */
+int32_t la_pbd_algo(const la_pbd_cfg* cfg, int32_t window_len);
 
 /*
  * Bytes of device workspace la_pbd_attn / la_pbd_step need for this configuration and window
@@ -133,7 +142,7 @@ la_status la_pbd_attn(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
 /*
  * One whole layer call: the result of la_kv_append followed by la_pbd_attn on the same
  * stream (same caches afterwards, same output bits). With the tcgen05 kernel (LA_ALGO_AUTO
- * with W * Hq/Hkv <= 64, or LA_ALGO_TCGEN05) both run in one launch: the attention kernel
+ * with W * Hq/Hkv <= 80, or LA_ALGO_TCGEN05) both run in one launch: the attention kernel
  * reads the window's keys and values from k_new / v_new and writes them into the caches
  * itself (the fused append; RK3588 model card, "How it differs from the original", item 1:
  * the window's rows are placed after the reused prefix, with no rollback). k_new and v_new
@@ -154,13 +163,17 @@ la_status la_pbd_step(const la_pbd_cfg* cfg, const void* q, const void* k_new,
  * Runs the same kernels as la_pbd_attn with their scratch in one file-scope device array of
  * 32 MiB that every GPU loading the library holds until the process exits; the call itself
  * allocates and frees nothing. Configurations whose la_pbd_workspace_bytes exceeds 32 MiB are
- * rejected with LA_ERR_WORKSPACE (nothing enqueued). The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. All calls on a device share the one array and it keeps the last
- * call's contents: calls whose executions overlap on the GPU (other streams, concurrent
- * threads) race on it and must be serialised by the caller. Device-side per-sequence errors
- * still produce zero rows, but their sticky flag stays in the shared array and is not readable
- * through la_pbd_check.
+ * rejected with LA_ERR_WORKSPACE (nothing enqueued); a valid configuration that cannot be
+ * sized because a device query failed gives LA_ERR_CUDA. Every call looks up the array's device
+ * address (cudaGetSymbolAddress) with the current device. Under CUDA's lazy module loading (the
+ * default since CUDA 12.2) the first call on each device loads the library's code there and
+ * reserves the array, which may allocate and synchronise: make that first call during set-up,
+ * outside any latency-critical loop, and before any stream capture. All calls on a device share
+ * the one array and it keeps the last call's contents: calls whose executions overlap on the
+ * GPU (other streams, concurrent threads) race on it and must be serialised by the caller.
+ * Nothing in it needs to start at zero (every value a kernel reads was written earlier in the
+ * same call). Device-side per-sequence errors still produce zero rows, but their sticky flag
+ * stays in the shared array and is not readable through la_pbd_check.
  */
 la_status la_pbd_attn_static(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                              const void* v_cache, const int32_t* seq_lens, int32_t window_len,
@@ -196,7 +209,7 @@ la_status la_pbd_step_varwin(const la_pbd_cfg* cfg, const void* q, const void* k
                              size_t workspace_bytes, void* stream);
 
 /*
- * Paged KV cache (tcgen05 kernel only, i.e. W * Hq/Hkv <= 64 and algo != LA_ALGO_SIMT, else
+ * Paged KV cache (tcgen05 kernel only, i.e. W * Hq/Hkv <= 80 and algo != LA_ALGO_SIMT, else
  * LA_ERR_UNSUPPORTED). The caches are page pools
  *   k_pool, v_pool  bf16 [num_pages, Hkv, page_size, D]
  *   block_table     device int32 [B, pages_per_seq]: key j of sequence b lives in page
@@ -230,7 +243,8 @@ la_status la_pbd_step_paged(const la_pbd_cfg* cfg, const void* q, const void* k_
  *   block_size     >= 1
  *   workspace      >= 256 bytes (its header, zeroed by la_pbd_workspace_init, receives the
  *                  sticky flags read by la_pbd_check)
- * bf16 inputs, fp32 accumulation, probabilities rounded to bf16 for the PV product, bf16 out.
+ * bf16 inputs, fp32 accumulation, bf16 out; the probabilities enter the PV product as two bf16
+ * parts (P_hi + P_lo), which keeps that product at fp32-level accuracy.
  * A sequence with T_b outside [0, min(t_max, S_max)] gets zero rows and the sticky flag.
  * Asynchronous on `stream`; allocates nothing.
  */
@@ -265,7 +279,8 @@ int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t window_len, const int32_t* se
                     int32_t max_segments);
 
 /*
- * Launch-floor helper: enqueue `launches` empty kernels of `ctas` x `threads` on `stream`,
+ * Measurement aid, not part of the attention path (the pages have no counterpart): the
+ * benchmark's launch-floor reference. Enqueues `launches` empty kernels of `ctas` x `threads` on `stream`,
  * chained with programmatic dependent launch like the library's own kernels. Timing a CUDA
  * graph of these beside a graph of real calls with the same launch count gives the part of
  * the step that launching alone costs. Asynchronous; allocates nothing. LA_ERR_INVALID_ARG
@@ -280,6 +295,23 @@ la_status la_noop_chain(int32_t launches, int32_t ctas, int32_t threads, void* s
  * Host only. LA_ERR_INVALID_ARG for another algo or a null pointer.
  */
 la_status la_pbd_plan_params(int32_t algo, int32_t* unit_keys, int32_t* seg_units);
+
+/*
+ * Self-test of the device-side failure detection (the pages have no counterpart). Every wait
+ * of the tensor-core kernels is bounded: when one runs out, the CTA raises the sticky
+ * LA_ERR_TIMEOUT flag in the workspace header, the kernel's other roles stop at their next
+ * wait, copies and tensor-core products in flight are drained with bounded waits, tensor
+ * memory is freed and the kernel returns, so the context stays usable. This call enqueues one
+ * la_pbd_attn on the tcgen05 kernel (the configuration must select it) in which every wait
+ * gives up after `wait_limit_ns` (1000 .. 2e9 ns) and the MMA thread withholds the completion
+ * signal of its first S^T product, so that the softmax warps' wait for it runs out. The call's
+ * `out` is then undefined; la_pbd_check afterwards returns LA_ERR_TIMEOUT and clears it, and
+ * the workspace serves the next call as usual. Arguments and errors otherwise as la_pbd_attn.
+ */
+la_status la_pbd_selftest_timeout(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* seq_lens,
+                                  int32_t window_len, void* out, void* workspace,
+                                  size_t workspace_bytes, int64_t wait_limit_ns, void* stream);
 
 /*
  * Synchronise `stream`, read and clear the workspace's sticky device-side error flags.

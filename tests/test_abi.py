@@ -59,7 +59,7 @@ def _cfg(**kw):
     (dict(num_kv_heads=1), 16, 2),         # W * G = 256 > 128
     (dict(mask_mode=7), 6, 1),
     (dict(algo=9), 6, 1),
-    (dict(algo=1, num_kv_heads=1), 5, 2),  # tensor-core kernel needs W * G <= 64
+    (dict(algo=1, num_kv_heads=1), 6, 2),  # tensor-core kernel needs W * G <= 80
     (dict(max_seq=0), 6, 1),
     (dict(batch=4096, num_kv_heads=16, num_q_heads=16, max_seq=1 << 20), 6, 2),
 ])
@@ -107,3 +107,21 @@ def test_noop_chain_validates_before_launching(lib):
     assert lib.la_noop_chain(4, 1, 0, None) == 1
     assert lib.la_noop_chain(4, 1, 1025, None) == 1
     assert lib.la_noop_chain(0, 1, 32, None) == 0     # nothing to launch
+
+
+def test_selftest_timeout_validates_before_launching(lib):
+    cfg = _cfg()
+    # wait limits outside [1 us, 2 s] are rejected before any CUDA call
+    for limit in (0, 999, 3_000_000_000):
+        assert lib.la_pbd_selftest_timeout(ctypes.byref(cfg), 16, 16, 16, 16, 6, 16, 256, 1 << 30,
+                                           limit, None) == 1
+
+
+def test_algo_choice_without_gpu(lib):
+    # kernel choice is host logic: tcgen05 up to 80 rows per KV head, CUDA cores above
+    assert bmw.la_pbd_algo(_cfg(), 6) == bmw.LA_ALGO_TCGEN05
+    assert bmw.la_pbd_algo(_cfg(), 10) == bmw.LA_ALGO_TCGEN05
+    assert bmw.la_pbd_algo(_cfg(), 11) == bmw.LA_ALGO_SIMT
+    assert bmw.la_pbd_algo(_cfg(algo=bmw.LA_ALGO_SIMT), 6) == bmw.LA_ALGO_SIMT
+    assert lib.la_pbd_algo(ctypes.byref(_cfg()), 17) == -1
+    assert lib.la_pbd_algo(ctypes.byref(_cfg(algo=1)), 11) == -2

@@ -1,0 +1,69 @@
+"""GPU test of the device-side failure detection: a bounded wait that runs out.
+
+Every wait of the tensor-core kernels is bounded. la_pbd_selftest_timeout runs one attention
+call in which the MMA thread withholds the completion signal of its first S^T product, with
+every wait limited to 1 ms: nothing else ever completes that barrier, so the softmax warps'
+wait for it runs out. No trap, fault or endless loop is involved. The kernel must raise the
+sticky LA_ERR_TIMEOUT flag, drain what it has in flight, free its tensor memory and return.
+The test checks the status, that it arrives quickly, and that the context, the tensor memory of
+the SMs that ran it and the same workspace then serve normal calls that match the oracle.
+"""
+import time
+
+import pytest
+import torch
+
+import block_masked_window_b200 as bmw
+import workloads
+from gpu_util import assert_parity, oracle_step, to_dev
+
+pytestmark = pytest.mark.gpu
+
+LA_ERR_TIMEOUT = 6
+
+
+def test_bounded_wait_runs_out_and_context_recovers(cuda_lib):
+    wl = workloads.WORKLOADS["tiny"]
+    wi = workloads.generate(wl)
+    li = wi.layers[0]
+    cfg = bmw.Config.make(wl.batch, wl.num_q_heads, wl.num_kv_heads, wi.max_seq,
+                          algo=bmw.LA_ALGO_TCGEN05)
+    q, kc, vc, sl = to_dev(li.q), to_dev(li.k_cache), to_dev(li.v_cache), to_dev(wi.seq_lens)
+    bmw.la_kv_append(cfg, to_dev(li.k_new), to_dev(li.v_new), kc, vc, sl, wl.window)
+    ws = bmw.Workspace(cfg, wl.window)
+    out = torch.full_like(q, float("nan"))
+    t0 = time.perf_counter()
+    bmw.la_pbd_selftest_timeout(cfg, q, kc, vc, sl, wl.window, out, ws, 1_000_000)
+    st = bmw.la_pbd_check(ws)
+    elapsed = time.perf_counter() - t0
+    assert st == LA_ERR_TIMEOUT, bmw.la_status_string(st)
+    assert elapsed < 5.0, elapsed
+    assert bmw.la_pbd_check(ws) == 0          # read and cleared
+
+    # The same workspace serves a normal call, whose result matches the oracle.
+    ref = oracle_step(li, wi.seq_lens, wl.scale)
+    out = torch.full_like(q, float("nan"))
+    bmw.la_pbd_attn(cfg, q, kc, vc, sl, wl.window, out, ws)
+    torch.cuda.synchronize()
+    assert bmw.la_pbd_check(ws) == 0
+    assert_parity(out.cpu(), ref, "after the timeout self-test")
+
+
+def test_every_sm_allocates_after_timeouts(cuda_lib):
+    """Timed-out CTAs on many SMs free their tensor memory: a full-grid call afterwards (one
+    CTA per SM, each allocating all 512 columns) completes and matches the oracle."""
+    wl = workloads.WORKLOADS["tiny"]
+    wi = workloads.random_case(40, [100 + 37 * i for i in range(40)], 6, seed=91)
+    li = wi.layers[0]
+    cfg = bmw.Config.make(40, 16, 2, wi.max_seq, algo=bmw.LA_ALGO_TCGEN05)
+    q, kc, vc, sl = to_dev(li.q), to_dev(li.k_cache), to_dev(li.v_cache), to_dev(wi.seq_lens)
+    bmw.la_kv_append(cfg, to_dev(li.k_new), to_dev(li.v_new), kc, vc, sl, 6)
+    ws = bmw.Workspace(cfg, 6)
+    out = torch.empty_like(q)
+    for _ in range(2):
+        bmw.la_pbd_selftest_timeout(cfg, q, kc, vc, sl, 6, out, ws, 1_000_000)
+        assert bmw.la_pbd_check(ws) == LA_ERR_TIMEOUT
+    bmw.la_pbd_attn(cfg, q, kc, vc, sl, 6, out, ws)
+    torch.cuda.synchronize()
+    assert bmw.la_pbd_check(ws) == 0
+    assert_parity(out.cpu(), oracle_step(li, wi.seq_lens, wi.workload.scale), "after timeouts")

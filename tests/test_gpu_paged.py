@@ -57,10 +57,11 @@ def gather(pool, table, seq_lens, W, S):
     return out
 
 
+@pytest.mark.parametrize("W", [6, 10])
 @pytest.mark.parametrize("page_size", [64, 128, 256])
 @pytest.mark.parametrize("mask_mode", [bmw.LA_MASK_PBD, bmw.LA_MASK_CAUSAL_WINDOW], ids=["pbd", "causal"])
-def test_paged_step(page_size, mask_mode):
-    prefixes, W = (0, 5, 121, 122, 1000, 2041, 300), 6
+def test_paged_step(page_size, mask_mode, W):
+    prefixes = (0, 5, 121, 122, 1000, 2041, 300)
     wi = workloads.random_case(len(prefixes), prefixes, W, seed=73)
     li = wi.layers[0]
     B, S = len(prefixes), wi.max_seq
@@ -84,7 +85,7 @@ def test_paged_step(page_size, mask_mode):
         assert np.array_equal(vg[b, :, :n].double().numpy(), v_ref[b, :, :n])
     mode = "causal" if mask_mode == bmw.LA_MASK_CAUSAL_WINDOW else "pbd"
     ref = oracle.window_attention(li.q, k_ref, v_ref, wi.seq_lens, wi.workload.scale, mask=mode)
-    assert_parity(out.cpu(), ref, f"paged page_size={page_size} {mode}")
+    assert_parity(out.cpu(), ref, f"paged page_size={page_size} {mode} W={W}")
 
 
 def test_paged_attn_matches_contiguous():

@@ -65,11 +65,16 @@ def test_small_prefixes(prefixes, W, algo):
     assert_parity(gpu, ref, f"P={prefixes} W={W}")
 
 
-@pytest.mark.parametrize("W", [9, 12, 16])
-def test_long_windows_simt(W):
-    wi = workloads.random_case(2, (40, 333), W, seed=7 + W)
+@pytest.mark.parametrize("algo", ALGOS + [bmw.LA_ALGO_AUTO], ids=ALGO_IDS + ["auto"])
+@pytest.mark.parametrize("W", [7, 8, 9, 10, 12, 16])
+def test_long_windows(W, algo):
+    """Windows of up to 10 rows (5 accepted tokens + 5 masks) on both kernels; the tcgen05
+    kernel takes W * G <= 80 rows (three S buffers and one P buffer from W = 9 at G = 8)."""
+    if algo == bmw.LA_ALGO_TCGEN05 and W * 8 > 80:
+        pytest.skip("the tcgen05 kernel takes W * G <= 80")
+    wi = workloads.random_case(3, (40, 333, 1300), W, seed=7 + W)
     li = wi.layers[0]
-    gpu = run_step(li, wi.seq_lens, wi.max_seq, W, algo=bmw.LA_ALGO_AUTO)
+    gpu = run_step(li, wi.seq_lens, wi.max_seq, W, algo=algo)
     ref = oracle_step(li, wi.seq_lens, wi.workload.scale)
     assert_parity(gpu, ref, f"W={W}")
 

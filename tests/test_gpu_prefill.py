@@ -1,12 +1,11 @@
 """GPU parity of the block-causal prefill kernel (la_block_prefill) against the fp64 oracle.
 
-Tolerance. The PV product takes the probabilities in bf16 (as flash attention does); the
-decode path splits them into two bf16 halves instead. Rounding P to bf16 adds a relative
-error of at most 2^-9 per probability, unbiased and independent between keys, which the
-decode measurements put at ~1.1e-3 relative L2 on N(0,1) data; the bf16 output rounding adds
-1.66e-3. Their root sum square is ~2.0e-3, so these tests bound the relative L2 error at
-3e-3 and the absolute error at 1e-2 (the decode path's max-abs bar), and do not apply the
-decode path's one-ulp check.
+Tolerance: the bar of the whole path, max |gpu - oracle| <= 1e-2 and relative L2 <= 2e-3
+(bf16 in, fp32 accumulate, bf16 out). The kernel splits the probabilities into two bf16 parts
+for the PV product (P = P_hi + P_lo, residual ~2^-17 P), as the decode path does, so the PV
+product adds nothing measurable to the bf16 output rounding (~1.7e-3 relative L2 on N(0,1)
+data). The decode path's extra one-ulp check is not applied: the prefill's 128-key tiles
+change the fp32 summation order over thousands of keys.
 """
 import numpy as np
 import pytest
@@ -20,7 +19,7 @@ from gpu_util import errors, to_dev
 pytestmark = pytest.mark.gpu
 
 MAX_ABS = 1e-2
-REL_L2 = 3e-3
+REL_L2 = 2e-3
 
 
 @pytest.fixture(scope="module", autouse=True)

@@ -36,16 +36,19 @@ def _case(prefixes, wlens, W_max, seed, Hq=16, Hkv=2):
 
 
 CASES = {
-    # (prefixes, window lengths, W_max): tcgen05 needs W_max * 8 <= 64
-    "tc": ((0, 5, 121, 1000, 2047, 300, 64, 250), (1, 8, 6, 7, 2, 8, 5, 3), 8),
-    "simt": ((0, 5, 121, 1000, 2047, 300, 64, 250), (1, 10, 6, 7, 2, 9, 5, 10), 10),
+    # (prefixes, window lengths, W_max); the pages' engine sends the accepted tokens (1..5)
+    # plus 5 masks, so W_b in [6, 10]; the tcgen05 kernel takes W_max * 8 <= 80
+    "w8": ((0, 5, 121, 1000, 2047, 300, 64, 250), (1, 8, 6, 7, 2, 8, 5, 3), 8),
+    "w10": ((0, 5, 121, 1000, 2047, 300, 64, 250), (1, 10, 6, 7, 2, 9, 5, 10), 10),
+    "w16": ((0, 5, 121, 1000), (16, 9, 3, 12), 16),
 }
 
 
 @pytest.mark.parametrize("mask_mode", [bmw.LA_MASK_PBD, bmw.LA_MASK_CAUSAL_WINDOW],
                          ids=["pbd", "causal"])
-@pytest.mark.parametrize("algo,key", [(bmw.LA_ALGO_TCGEN05, "tc"), (bmw.LA_ALGO_SIMT, "simt")],
-                         ids=["tcgen05", "simt"])
+@pytest.mark.parametrize("algo,key", [(bmw.LA_ALGO_TCGEN05, "w8"), (bmw.LA_ALGO_TCGEN05, "w10"),
+                                      (bmw.LA_ALGO_SIMT, "w10"), (bmw.LA_ALGO_SIMT, "w16")],
+                         ids=["tcgen05-w8", "tcgen05-w10", "simt-w10", "simt-w16"])
 def test_variable_windows(algo, key, mask_mode):
     prefixes, wlens, W_max = CASES[key]
     wi, li, q, kn, vn, wl = _case(prefixes, wlens, W_max, seed=51)
@@ -70,10 +73,11 @@ def test_variable_windows(algo, key, mask_mode):
         assert_parity(o[b, :w], ref[b, :w], f"varwin {key} {mode} b={b} W_b={w}")
 
 
-def test_variable_windows_fused_matches_separate():
+@pytest.mark.parametrize("key", ["w8", "w10"])
+def test_variable_windows_fused_matches_separate(key):
     """The tcgen05 step (append fused into the attention launch) against the CUDA-core step
     (append kernel, then attention): same caches bit for bit, outputs within rounding."""
-    prefixes, wlens, W_max = CASES["tc"]
+    prefixes, wlens, W_max = CASES[key]
     wi, li, q, kn, vn, wl = _case(prefixes, wlens, W_max, seed=53)
     B = len(prefixes)
     outs, caches = [], []

@@ -4,8 +4,11 @@ Callers such as an engine plugin that is handed no scratch memory, or a decode l
 cudaMalloc is forbidden (it can synchronise the device), use la_pbd_attn_static instead of
 la_pbd_attn: the library supplies the scratch from one 32 MiB device array per GPU. This test
 calls it through the C ABI twice in a row and checks each output against la_pbd_attn with a
-caller workspace, within the parity tolerance used by the other GPU tests. It lives in its own
-file, collected last, and passes alone in a fresh process as well as after the other tests.
+caller workspace and against the fp64 oracle, within the parity tolerance used by the other
+GPU tests. The single-image layer (one sequence, split over several CTAs) puts split partial
+results in the shared array; the ragged batch covers many sequences and the prefix sums the
+merge reads for batches above 32. It lives in its own file, collected last, and passes alone
+in a fresh process as well as after the other tests.
 """
 import ctypes
 
@@ -13,7 +16,9 @@ import pytest
 import torch
 
 import block_masked_window_b200 as bmw
+import oracle
 import workloads
+from gpu_util import errors
 
 pytestmark = pytest.mark.gpu
 
@@ -26,10 +31,11 @@ def _close(a, b):
     return float((a - b).abs().max()) <= MAX_ABS and float((a - b).norm() / b.norm()) <= REL_L2
 
 
+@pytest.mark.parametrize("workload", ["single_image", "ragged"])
 @pytest.mark.parametrize("algo", [bmw.LA_ALGO_TCGEN05, bmw.LA_ALGO_SIMT], ids=["tcgen05", "simt"])
-def test_static_entry_matches_workspace_entry(cuda_lib, algo):
-    wl = workloads.WORKLOADS["ragged"]
-    wi = workloads.generate(wl)
+def test_static_entry_matches_workspace_entry(cuda_lib, algo, workload):
+    wl = workloads.WORKLOADS[workload]
+    wi = workloads.generate(wl, layers=1)
     li = wi.layers[0]
     cfg = bmw.Config.make(wl.batch, wl.num_q_heads, wl.num_kv_heads, wi.max_seq, algo=algo)
     dev = lambda t: t.contiguous().cuda()  # noqa: E731
@@ -37,6 +43,8 @@ def test_static_entry_matches_workspace_entry(cuda_lib, algo):
     bmw.la_kv_append(cfg, dev(li.k_new), dev(li.v_new), kc, vc, sl, wl.window)
     ref = torch.empty_like(q)
     bmw.la_pbd_attn(cfg, q, kc, vc, sl, wl.window, ref, bmw.Workspace(cfg, wl.window))
+    exact = oracle.pbd_step(li.q, li.k_cache, li.v_cache, li.k_new, li.v_new, wi.seq_lens,
+                            wl.scale)
     lib = bmw.load()
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
@@ -47,6 +55,8 @@ def test_static_entry_matches_workspace_entry(cuda_lib, algo):
         torch.cuda.synchronize()
         assert torch.isfinite(out).all()
         assert _close(out.cpu(), ref.cpu())
+        max_abs, rel = errors(out.cpu(), exact)
+        assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
 
 
 def test_static_entry_rejects_oversized_problem(cuda_lib):
