@@ -124,8 +124,7 @@ __global__ void __launch_bounds__(kThreads) pbd_attn_simt_kernel(Problem p) {
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i <= p.B; i += blockDim.x) p.pre_g[i] = s.pre[i];
   }
-  const long long C = plan_chunk(p, T);
-  SegmentIter it = plan_begin(p, s.pre, blockIdx.x, C, T);
+  SegmentIter it = plan_begin(p, s.pre, blockIdx.x, T);
 
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int hf = lane >> 4, tl = lane & 15;

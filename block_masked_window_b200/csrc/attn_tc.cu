@@ -358,13 +358,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     const int excl = incl - u;
     const long long Tg = (long long)p.Hkv * __shfl_sync(0xffffffffu, incl, 31);
-    const long long Cg = Tg > 0 ? plan_chunk(p, Tg) : 1;
-    const long long pos = (long long)blockIdx.x * Cg;
+    const long long pos = Tg > 0 ? plan_lo(p, Tg, blockIdx.x) : 0;
+    const long long Cg = Tg > 0 ? plan_lo(p, Tg, blockIdx.x + 1) - pos : 0;   // units of this CTA
     const unsigned starts = __ballot_sync(0xffffffffu, lane < p.B && u > 0 &&
                                                            (long long)p.Hkv * excl <= pos);
     const int bb = starts ? 31 - __clz(starts) : 0;
     const int ub = __shfl_sync(0xffffffffu, u, bb), pb = __shfl_sync(0xffffffffu, excl, bb);
-    if (lane == 0 && pos < Tg && starts != 0u && ub > 0) {
+    if (lane == 0 && Cg > 0 && starts != 0u && ub > 0) {
       const long long off = pos - (long long)p.Hkv * pb;
       const int hh = (int)(off / ub);
       const int t0 = max((int)(off - (long long)hh * ub) - p.seg_units, 0);  // first key tile
@@ -387,6 +387,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   // once every CTA is past the wait (it reads seq_lens before its own wait).
   pdl_wait();
   pdl_trigger();
+  if (tid == 0) {
+    // The tensor maps' descriptors again, now that the wait is over (the copies of the first
+    // tiles are issued right after the plan).
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmq)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+  }
   plan_prefix(p, pre, warp_tot);
   fence_async_smem();
   tc_fence_before();
@@ -398,12 +405,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   if (blockIdx.x == 0) {
     for (int i = tid; i <= p.B; i += kThreadsTc) p.pre_g[i] = pre[i];
   }
-  const long long C = plan_chunk(p, T);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer: Q, K
     // Lane 0 issues the copies; the whole warp moves the window rows of a fused append.
-    SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
+    SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
     Segment sg;
     int g = 0, nseg = 0;
     uint32_t raw_par = 0;   // phase parity of each stage's fused-append barrier
@@ -470,7 +476,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------------ TMA producer: V
-    SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
+    SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
     Segment sg;
     int g = 0;
     uint32_t raw_par = 0;
@@ -522,7 +528,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
+      SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
       Segment sg;
       int g = 0, nseg = 0;
       bool ok = true;
@@ -634,7 +640,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     float* rowst = reinterpret_cast<float*>(base + L.mref);   // [2][NQ]
     float* alpha_s = reinterpret_cast<float*>(base + L.alpha); // [NQ]
     const float c2 = p.scale_log2;
-    SegmentIter it = plan_begin(p, pre, blockIdx.x, C, T);
+    SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
     Segment sg;
     int g = 0;
     bool ok = true;

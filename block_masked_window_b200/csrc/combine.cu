@@ -9,7 +9,10 @@
 //
 // One warp per output row (4 rows per 128-thread block): lane k holds partial k's maximum and
 // sum, the warp reduces them (weights kept in shared memory), and each lane accumulates 4 of
-// the 128 channels over the partials with independent 16-byte loads.
+// the 128 channels over the partials with independent 16-byte loads. The first KM partial rows
+// are loaded in one round trip with the maxima and sums: KM = 16, or 40 where a sequence can
+// be split into more than 16 pieces at a small batch (one sequence over up to 40 CTAs, e.g. a
+// 4096-token prefix at one tile per CTA), where a second round trip would otherwise follow.
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 
@@ -17,8 +20,7 @@ namespace la {
 
 constexpr int kCombineRows = 4;
 constexpr int kCombineMaxSlots = 1024;   // >= partials of one sequence (<= grid size)
-constexpr int kMerge = 16;               // partials loaded in the first round trip
-
+template <int kMerge>   // partials loaded in the first round trip
 __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem p) {
   __shared__ float s_w[kCombineRows][kCombineMaxSlots];
   pdl_trigger();
@@ -62,13 +64,12 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
   if (r >= p.R) return;
   __nv_bfloat16* dst = p.out + out_row_offset(p, b, h, r);
   const long long T = (long long)p.Hkv * ptot;
-  const long long C = plan_chunk(p, T);
   const long long off = (long long)p.Hkv * pb + (long long)h * u;
   if (u > 0 && r / p.G >= wb) {
     // Padding row of a shorter window: written as zeros by whichever kernel owns the
     // sequence (here if it was split; the attention kernel if it was whole).
     int f0, l0;
-    plan_tile_ctas(p, off, u, C, &f0, &l0);
+    plan_tile_ctas(p, off, u, T, &f0, &l0);
     if (f0 != l0) reinterpret_cast<uint2*>(dst)[lane] = make_uint2(0u, 0u);
     return;
   }
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
     return;
   }
   int c0, c1;
-  plan_tile_ctas(p, off, u, C, &c0, &c1);
+  plan_tile_ctas(p, off, u, T, &c0, &c1);
   if (c0 == c1) return;
   const int ns = c1 - c0 + 1;
   const size_t stride = slot_floats(p.rows_pad);
@@ -92,19 +93,27 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
 #pragma unroll
   for (int u = 0; u < kMerge; ++u)
     if (u < ns) a[u] = *reinterpret_cast<const float4*>(acc0 + (size_t)u * stride);
-  float mk = -INFINITY, lk = 0.f;
+  // Maxima and sums of partials lane and lane + 32, in the same round trip (up to 64
+  // partials; more take further round trips).
+  float mk0 = -INFINITY, lk0 = 0.f, mk1 = -INFINITY, lk1 = 0.f;
   if (lane < ns) {
-    mk = base[(size_t)lane * stride + r];
-    lk = base[(size_t)lane * stride + p.rows_pad + r];
+    mk0 = base[(size_t)lane * stride + r];
+    lk0 = base[(size_t)lane * stride + p.rows_pad + r];
   }
-  float M = mk;
-  for (int k = lane + 32; k < ns; k += 32) M = fmaxf(M, base[(size_t)k * stride + r]);
+  if (lane + 32 < ns) {
+    mk1 = base[(size_t)(lane + 32) * stride + r];
+    lk1 = base[(size_t)(lane + 32) * stride + p.rows_pad + r];
+  }
+  float M = fmaxf(mk0, mk1);
+  for (int k = lane + 64; k < ns; k += 32) M = fmaxf(M, base[(size_t)k * stride + r]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float wk = (mk == -INFINITY) ? 0.f : fast_exp2(mk - M);
-  if (lane < ns) s_w[warp][lane] = wk;
-  float L = wk * lk;
-  for (int k = lane + 32; k < ns; k += 32) {
+  const float w0 = (mk0 == -INFINITY) ? 0.f : fast_exp2(mk0 - M);
+  const float w1 = (mk1 == -INFINITY) ? 0.f : fast_exp2(mk1 - M);
+  if (lane < ns) s_w[warp][lane] = w0;
+  if (lane + 32 < ns) s_w[warp][lane + 32] = w1;
+  float L = fmaf(w0, lk0, w1 * lk1);
+  for (int k = lane + 64; k < ns; k += 32) {
     const float m2 = base[(size_t)k * stride + r];
     const float w2 = (m2 == -INFINITY) ? 0.f : fast_exp2(m2 - M);
     s_w[warp][k] = w2;
@@ -145,7 +154,14 @@ __global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem 
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream) {
   if (p.num_ctas > kCombineMaxSlots) return cudaErrorInvalidValue;
   dim3 grid((p.R + kCombineRows - 1) / kCombineRows, p.B * p.Hkv);
-  return launch_pdl(pbd_combine_kernel, grid, dim3(32 * kCombineRows), 0, stream, p);
+  // A sequence is split into at most one piece per key tile of its capacity, and (with C >= 1
+  // units per CTA) at most one per CTA; the larger first batch pays off only where that bound
+  // exceeds 16 and the batch is small enough for the merge to be latency-bound.
+  const long long tiles = (p.S + p.unit - 1) / p.unit;
+  const long long pieces = tiles < p.num_ctas ? tiles : p.num_ctas;
+  if (pieces > 16 && (long long)p.B * p.Hkv <= 4)
+    return launch_pdl(pbd_combine_kernel<40>, grid, dim3(32 * kCombineRows), 0, stream, p);
+  return launch_pdl(pbd_combine_kernel<16>, grid, dim3(32 * kCombineRows), 0, stream, p);
 }
 
 }  // namespace la

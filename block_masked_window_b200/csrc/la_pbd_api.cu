@@ -308,10 +308,9 @@ int32_t la_pbd_plan(const la_pbd_cfg* cfg, int32_t W, const int32_t* seq_lens_ho
   std::vector<int> pre(p.B + 1, 0);
   for (int b = 0; b < p.B; ++b) pre[b + 1] = pre[b] + la::plan_units_of(p, la::visible_len(p, b));
   const long long T = (long long)p.Hkv * pre[p.B];
-  const long long C = la::plan_chunk(p, T);
   int32_t count = 0;
   for (int c = 0; c < num_ctas; ++c) {
-    la::SegmentIter it = la::plan_begin(p, pre.data(), c, C, T);
+    la::SegmentIter it = la::plan_begin(p, pre.data(), c, T);
     la::Segment sg;
     while (it.next(p, pre.data(), c, sg)) {
       if (count < max_segments) {

@@ -5,9 +5,11 @@
 // N_b = P_b + W visible keys (0 if P_b is invalid), cut into U_b = ceil(N_b / unit) units of
 // `unit` keys (the attention kernel's key tile; only a sequence's last unit is partial). All
 // sequences are laid end to end in one flattened stream of T = Hkv * sum_b U_b units. CTA c
-// of a grid of G CTAs owns units [c*C, (c+1)*C) with C = max(c_min, ceil(T / G)), so every
-// CTA gets the same number of whole tiles whatever the mix of prefix lengths, and no tile is
-// ever shared by two CTAs. The part of a sequence that falls in one CTA is a segment; a CTA
+// of a grid of G CTAs owns units [lo(c), lo(c + 1)) with lo(c) = floor(c * T / G) when
+// T >= G, so every CTA gets floor(T / G) or ceil(T / G) whole tiles (at least one) whatever
+// the mix of prefix lengths; when T < G, CTA c takes unit c alone. No tile is ever shared by
+// two CTAs, and every CTA between the first and the last of a sequence holds a piece of it.
+// The part of a sequence that falls in one CTA is a segment; a CTA
 // that holds a whole sequence writes its final output directly, every other segment writes
 // an (m, l, acc) partial to slot c + s, and the combine kernel merges them. Slot c + s is
 // unique because CTAs and sequences advance together along the stream.
@@ -167,10 +169,18 @@ __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
   }
 }
 
-// Chunk size C from the total T (identical in every kernel that uses the plan).
-__host__ __device__ inline long long plan_chunk(const Problem& p, long long T) {
-  long long c = (T + p.num_ctas - 1) / p.num_ctas;
-  return c < p.c_min ? (long long)p.c_min : c;
+// First unit of CTA c (c in [0, num_ctas]) for a stream of T units (identical in every kernel
+// that uses the plan): floor(c * T / G) when T >= G, else min(c, T).
+__host__ __device__ inline long long plan_lo(const Problem& p, long long T, int c) {
+  if (T < p.num_ctas) return c < T ? (long long)c : T;
+  return (long long)c * T / p.num_ctas;
+}
+
+// The CTA that owns unit x (0 <= x < T): the largest c with plan_lo(c) <= x, i.e.
+// c * T < (x + 1) * G when T >= G, else x.
+__host__ __device__ inline int plan_cta_of(const Problem& p, long long T, long long x) {
+  if (T < p.num_ctas) return (int)x;
+  return (int)(((x + 1) * p.num_ctas - 1) / T);
 }
 
 // Largest b with Hkv * pre[b] <= pos (pos < T). Never returns a zero-length sequence.
@@ -226,19 +236,18 @@ struct SegmentIter {
 };
 
 // CTAs that hold the first and the last key tile of (b, h), whose units start at s0 = off
-// and number u > 0 (chunk size C): the sequence is split iff they differ, and its partial
+// and number u > 0 (stream of T units): the sequence is split iff they differ, and its partial
 // results sit in slots c + b * Hkv + h for c in [first, last].
-__host__ __device__ inline void plan_tile_ctas(const Problem& p, long long off, int u, long long C,
+__host__ __device__ inline void plan_tile_ctas(const Problem& p, long long off, int u, long long T,
                                                int* first, int* last) {
-  *first = (int)((off + p.seg_units) / C);
-  *last = (int)((off + u - 1) / C);
+  *first = plan_cta_of(p, T, off + p.seg_units);
+  *last = plan_cta_of(p, T, off + u - 1);
 }
 
-__host__ __device__ inline SegmentIter plan_begin(const Problem& p, const int* pre, int c, long long C,
-                                         long long T) {
+__host__ __device__ inline SegmentIter plan_begin(const Problem& p, const int* pre, int c, long long T) {
   SegmentIter it;
-  it.pos = (long long)c * C;
-  it.end = it.pos + C < T ? it.pos + C : T;
+  it.pos = plan_lo(p, T, c);
+  it.end = plan_lo(p, T, c + 1);
   it.b = 0; it.h = 0;
   if (it.pos < T) {
     int b = plan_find_batch(p, pre, it.pos);

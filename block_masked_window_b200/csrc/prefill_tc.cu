@@ -16,13 +16,15 @@
 // softmax threads own query row r (TMEM lane r), one per key half: each reads its 64 scores
 // from TMEM, keeps its lazy reference maximum (raised only when a score exceeds it by 2^8;
 // the warp then rescales its O_h rows after the previous PV product has completed) and row
-// sum in registers, and writes its half of the row of P into shared memory in the
-// 128-byte-swizzled K-major layout the MMA reads. P is written as two bf16 parts, P = P_hi +
-// P_lo (P_lo = bf16(P - P_hi), residual ~2^-17 P), and each PV product is issued for both
-// parts, so the product keeps fp32-level accuracy in P: a single bf16 rounding of P would add
-// a relative L2 error of ~1e-3 to the output, on top of the ~1.7e-3 of its own bf16 rounding.
-// The P region of a key half is single-buffered: the softmax of tile t computes its
-// probabilities first and waits for the PV product of tile t - 1 only before storing them.
+// sum in registers, and writes its half of the row of P back into tensor memory, over the
+// 64 score columns it has just read: P is written as two bf16 parts, P = P_hi + P_lo (P_lo =
+// bf16(P - P_hi), residual ~2^-17 P), packed two keys per column (P_hi in the first 32
+// columns, P_lo in the next 32), and each PV product is issued for both parts with A read
+// from tensor memory, so the product keeps fp32-level accuracy in P: a single bf16 rounding
+// of P would add a relative L2 error of ~1e-3 to the output, on top of the ~1.7e-3 of its own
+// bf16 rounding. P lives in the S buffer of its tile, so it is double-buffered with S, and
+// shared memory holds only Q and the K and V rings (three stages each). The product S of
+// tile t + 2 reuses that buffer once both halves' PV products of tile t have completed.
 // With no exchange between the halves per tile, the two warps sharing a scheduler drift
 // apart, so one's exponentials overlap the other's maxima and TMEM reads. At the end the pair
 // merges (m, l, O_0, O_1) and each thread normalises and stores 64 of the row's 128 output
@@ -46,13 +48,12 @@ using namespace tc;
 constexpr int kBM = 128;                 // query rows per CTA
 constexpr int kBN = 128;                 // keys per tile
 constexpr int kPfThreads = 352;         // 11 warps
-constexpr int kPfStages = 2;             // K and V ring depth
+constexpr int kPfStages = 3;             // K and V ring depth
 constexpr int kPHalf = 128 * 128;        // one 64-column half of a 128-row bf16 tile (16 KB)
-constexpr int kPTile = 2 * kPHalf;       // 32 KB
-constexpr int kPRegion = 2 * kPHalf;     // P of one key half: P_hi (16 KB) then P_lo (16 KB)
+constexpr int kPTile = 2 * kPHalf;       // 32 KB: a 128-row x 128-channel bf16 operand tile
 constexpr float kPfLazy = 8.f;           // log2 units
 constexpr int kPfTmemCols = 512;
-constexpr int kColS = 0;                 // S: 2 buffers x 128 columns
+constexpr int kColS = 0;                 // S (then P_hi | P_lo per key half): 2 buffers x 128
 constexpr int kColO = 2 * kBN;           // O of key half 0 (128 columns), then of key half 1
 
 constexpr int kBQFull = 0;
@@ -66,12 +67,11 @@ constexpr int kBOFull = kBPFull + 4;              // [key half][tile parity]
 constexpr int kBDrain = kBOFull + 4;
 constexpr int kBNum = kBDrain + 1;
 
-// Shared memory: Q | K ring | V ring | P (two key halves x {P_hi, P_lo}) | barriers | misc.
+// Shared memory: Q | K ring | V ring | barriers | misc.
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kPTile;
 constexpr int kOffV = kOffK + kPfStages * kPTile;
-constexpr int kOffP = kOffV + kPfStages * kPTile;
-constexpr int kOffBar = kOffP + 2 * kPRegion;
+constexpr int kOffBar = kOffV + kPfStages * kPTile;
 constexpr int kOffMisc = kOffBar + kBNum * 8;
 constexpr int kPfSmem = kOffMisc + 16;
 // The final (m, l) exchange of the two halves ([2][2 halves][128 rows] floats) reuses the Q
@@ -82,12 +82,12 @@ constexpr size_t kPfSmemAlloc = (size_t)kPfSmem + 1024;   // + alignment slack
 // Named barrier 1 over the 256 softmax threads.
 __device__ __forceinline__ void pf_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-// 8 probabilities (keys 8 k8 .. 8 k8 + 7 of a key half) of row r as bf16 P_hi and P_lo into
-// the swizzled K-major P region of that half; `prow` is row r of its P_hi part.
-__device__ __forceinline__ void store_p_hilo(uint32_t prow, int k8, int r, const float* x) {
-  uint32_t hi[4], lo[4];
+// The 64 probabilities of one key half of a row as bf16 P_hi and P_lo, two keys per 32-bit
+// word (the lower key in the low half), into 32 + 32 tensor-memory columns from `taddr`.
+__device__ __forceinline__ void store_p_tmem(uint32_t taddr, const float (&x)[64]) {
+  uint32_t hi[32], lo[32];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
+  for (int e = 0; e < 32; ++e) {
     const float a = x[2 * e], b = x[2 * e + 1];
     __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
     hi[e] = *reinterpret_cast<uint32_t*>(&h2);
@@ -95,11 +95,8 @@ __device__ __forceinline__ void store_p_hilo(uint32_t prow, int k8, int r, const
     __nv_bfloat162 l2 = __floats2bfloat162_rn(a - ha, b - hb);
     lo[e] = *reinterpret_cast<uint32_t*>(&l2);
   }
-  const uint32_t a = prow + (uint32_t)(((k8 ^ (r & 7)) << 4));
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(hi[0]), "r"(hi[1]),
-               "r"(hi[2]), "r"(hi[3]));
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a + kPHalf), "r"(lo[0]),
-               "r"(lo[1]), "r"(lo[2]), "r"(lo[3]));
+  tmem_st32(taddr, hi);
+  tmem_st32(taddr + 32, lo);
 }
 
 }  // namespace
@@ -110,7 +107,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   extern __shared__ __align__(1024) char smem_raw[];
   char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(base);
-  const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV, sP = sb + kOffP;
+  const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV;
   auto bar = [&](int i) { return sb + (uint32_t)kOffBar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 8);
@@ -211,7 +208,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_f16(128, kBN, 0, 0);     // Q K-major, K K-major
-      constexpr uint32_t kIdO = idesc_f16(128, 128, 0, 1);     // P K-major, V MN-major
+      constexpr uint32_t kIdO = idesc_f16(128, 128, 0, 1);     // P (tensor memory), V MN-major
       bool ok = mbar_wait(bar(kBQFull), 0, ctl);
       tc_fence_after();
       int nqk = 0, npv[2] = {0, 0};
@@ -219,10 +216,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t spins = 0;
       while (ok && (npv[0] < nk || npv[1] < nk)) {
         bool prog = false;
-        // S(t) into buffer t & 1 once both halves have read S(t - 2) (their PV(t - 2) issued).
+        // S(t) into buffer t & 1 once both halves' PV(t - 2) products, which read P(t - 2)
+        // from that buffer, have completed.
         if (nqk < nk && nqk <= min(npv[0], npv[1]) + 1) {
           const int s = nqk % kPfStages;
-          if (mbar_test(bar(kBKFull + s), (nqk / kPfStages) & 1)) {
+          const int tp = nqk - 2;
+          const bool sfree = tp < 0 || (mbar_test(bar(kBOFull + (tp & 1)), (tp >> 1) & 1) &&
+                                        mbar_test(bar(kBOFull + 2 + (tp & 1)), (tp >> 1) & 1));
+          if (sfree && mbar_test(bar(kBKFull + s), (nqk / kPfStages) & 1)) {
             tc_fence_after();
             const uint32_t d = tmem + kColS + (uint32_t)((nqk & 1) * kBN);
             const uint32_t kb = sK + s * kPTile;
@@ -248,14 +249,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (mbar_test(bar(kBPFull + 2 * hh + (t & 1)), (t >> 1) & 1) &&
                 mbar_test(bar(kBVFull + s), (t / kPfStages) & 1)) {
               tc_fence_after();
-              const uint32_t pb = sP + hh * kPRegion;
+              const uint32_t pa = tmem + kColS + (uint32_t)((t & 1) * kBN + 64 * hh);   // P_hi
               const uint32_t vb = sV + s * kPTile + hh * 4 * 2048;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t vd = sdesc(vb + kk * 2048, kPHalf, 1024, 2);
-                umma(tmem + kColO + hh * 128, sdesc(pb + kk * 32, 16, 1024, 2), vd, kIdO,
-                     (t > 0 || kk > 0) ? 1u : 0u);
-                umma(tmem + kColO + hh * 128, sdesc(pb + kPHalf + kk * 32, 16, 1024, 2), vd, kIdO, 1u);
+                umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+                umma_ts(tmem + kColO + hh * 128, pa + 32 + kk * 8, vd, kIdO, 1u);
               }
               umma_commit(bar(kBOFull + 2 * hh + (t & 1)));
               ++npv[hh];
@@ -358,15 +358,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ls[e & 3] += x[e];
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // This half's P region was last read by this half's PV product of the previous tile.
-      if (t > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(kBOFull + 2 * half + ((t - 1) & 1)), ((t - 1) >> 1) & 1, ctl))) { ok = false; break; }
-        tc_fence_after();
-      }
-      // P_hi and P_lo into this half's swizzled K-major P rows, 8 keys per 16-byte store each.
-      const uint32_t prow = sP + half * kPRegion + (uint32_t)r * 128u;
-#pragma unroll
-      for (int k8 = 0; k8 < 8; ++k8) store_p_hilo(prow, k8, r, x + 8 * k8);
+      // P_hi and P_lo over this half's scores in the S buffer of the tile (read above).
+      store_p_tmem(s_addr, x);
+      tc_wait_st();
       // Keys of this half past the visible range (last tile): zero their V rows so that
       // 0 * x cannot become NaN in the product (those rows may hold anything).
       const int valid = min(kBN, kmax - t * kBN);

@@ -155,3 +155,25 @@ def test_plan_rejects_bad_arguments():
             bmw.la_pbd_plan(cfg, 6, [1, 2], num_ctas, unit, seg)
     with pytest.raises(bmw.LaError):
         bmw.la_pbd_plan(bmw.Config.make(2, 16, 3, 128), 6, [1, 2], 4, 128)
+
+
+def test_plan_spreads_units_over_every_cta():
+    """With at least as many units as CTAs, every CTA gets floor(T/G) or ceil(T/G) of them, so
+    on the ragged batch all 148 CTAs get work (a uniform chunk of ceil(T/G) left the last
+    CTAs idle); with fewer units than CTAs the units go one per CTA from CTA 0, so the pieces
+    of a sequence stay in consecutive CTAs."""
+    gen = torch.Generator().manual_seed(3)
+    base = torch.randint(512, 4096 + 1, (64,), generator=gen, dtype=torch.int64)
+    acc = torch.randint(1, 5 + 1, (64,), generator=gen, dtype=torch.int64)
+    lens = (base + acc).tolist()
+    unit, seg = bmw.la_pbd_plan_params(bmw.LA_ALGO_TCGEN05)
+    segs = check_plan(lens, 6, 4160, 2, 148, unit, seg=seg)
+    assert {s[0] for s in segs} == set(range(148))
+    T = sum(2 * (-(-(P + 6) // unit) + seg) for P in lens)
+    units = {}
+    for cta, b, h, j0, j1, slot in segs:
+        units[cta] = units.get(cta, 0) + -(-(j1 - j0) // unit)
+    # tiles alone never exceed the share; the fixed costs fill the rest of it
+    assert max(units.values()) <= -(-T // 148)
+    segs = check_plan([1024], 6, 1088, 2, 148, unit)     # 18 tiles on 148 CTAs
+    assert sorted(s[0] for s in segs) == list(range(18))

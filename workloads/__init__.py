@@ -89,6 +89,9 @@ WORKLOADS = {
 }
 # NTP fallback on the max-context caches (same seed, same max_seq, window 1).
 WORKLOADS["max_context_w1"] = WORKLOADS["max_context"].with_window(1)
+# The longest window the RKLLM engine sends (5 accepted tokens + 5 <text_mask> tokens, RK3588
+# model card, item 1) on the ragged batch: a timing case for the kernel choice at 80 rows.
+WORKLOADS["ragged_w10"] = WORKLOADS["ragged"].with_window(10)
 
 ORDER = ["tiny", "single_image", "max_context", "max_context_w1", "ragged", "long"]
 
