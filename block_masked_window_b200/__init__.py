@@ -18,7 +18,7 @@ __all__ = [
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
     "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
     "la_noop_chain", "la_pbd_attn_varwin", "la_pbd_algo", "chosen_algo",
-    "la_pbd_selftest_timeout",
+    "la_pbd_selftest_timeout", "la_pbd_selftest_replan",
     "la_pbd_step_varwin", "la_block_prefill", "la_pbd_attn_paged", "la_pbd_step_paged",
     "Workspace",
     "EXPORTED_SYMBOLS",
@@ -40,6 +40,7 @@ EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
                     "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
                     "la_noop_chain", "la_pbd_algo", "la_pbd_selftest_timeout",
+                    "la_pbd_selftest_replan",
                     "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill",
                     "la_pbd_attn_paged", "la_pbd_step_paged"]
 
@@ -122,6 +123,8 @@ def load() -> ctypes.CDLL:
     lib.la_noop_chain.argtypes = [i32, i32, i32, vp]
     lib.la_pbd_algo.restype = i32
     lib.la_pbd_algo.argtypes = [cfgp, i32]
+    lib.la_pbd_selftest_replan.restype = i32
+    lib.la_pbd_selftest_replan.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.la_pbd_selftest_timeout.restype = i32
     lib.la_pbd_selftest_timeout.argtypes = [cfgp, vp, vp, vp, vp, i32, vp, vp, sz, ctypes.c_int64,
                                             vp]
@@ -310,6 +313,27 @@ def la_pbd_selftest_timeout(cfg: Config, q, k_cache, v_cache, seq_lens, window_l
                                           workspace.data_ptr(), workspace.nbytes,
                                           int(wait_limit_ns), _stream(stream)),
            "la_pbd_selftest_timeout")
+
+
+def la_pbd_selftest_replan(cfg: Config, q, k_new, v_new, k_cache, v_cache, seq_lens,
+                           window_len: int, out, workspace: Workspace, stream=None) -> None:
+    """Enqueue la_pbd_attn (k_new, v_new None) or la_pbd_step with the plan made before the
+    dependency wait forced to be rejected (self-test of the kernel's re-plan path)."""
+    W = int(window_len)
+    q_shape, cache_shape, new_shape = _shapes(cfg, W)
+    _check_tensor(q, "q", "bf16", q_shape)
+    if k_new is not None:
+        _check_tensor(k_new, "k_new", "bf16", new_shape)
+        _check_tensor(v_new, "v_new", "bf16", new_shape)
+    _check_tensor(k_cache, "k_cache", "bf16", cache_shape)
+    _check_tensor(v_cache, "v_cache", "bf16", cache_shape)
+    _check_tensor(seq_lens, "seq_lens", "i32", (cfg.batch,))
+    _check_tensor(out, "out", "bf16", q_shape)
+    _check(load().la_pbd_selftest_replan(ctypes.byref(cfg), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                         _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), W,
+                                         _ptr(out), workspace.data_ptr(), workspace.nbytes,
+                                         _stream(stream)),
+           "la_pbd_selftest_replan")
 
 
 def la_pbd_algo(cfg: Config, window_len: int) -> int:

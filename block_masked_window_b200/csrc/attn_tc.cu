@@ -121,8 +121,8 @@ __host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, in
   L.lim = a16(L.wmax + 2 * 4 * nq * 4);     // [3][nq] ints: (unused), output offsets, key limits
   L.mref = a16(L.lim + 3 * nq * 4);         // [2][nq]: per-row references
   L.alpha = a16(L.mref + 2 * nq * 4);       // [nq]: rescale factors of the last reference update
-  L.pre = a16(L.alpha + nq * 4);            // [B+1] + 32 ints
-  L.end = L.pre + (round_up(B + 1, 4) + 32) * 4;
+  L.pre = a16(L.alpha + nq * 4);            // plan: [B+1] twice, 32 ints, first segment (16 x 8 B)
+  L.end = L.pre + (2 * round_up(B + 1, 4) + 32) * 4 + 16 * 8;
   return L;
 }
 
@@ -181,15 +181,16 @@ __device__ __forceinline__ int kv_row(const Problem& p, int b, int h, int j) {
 // Issues the two (contiguous) or four (paged: one 64-row box per page piece) TMA loads of key
 // tile [jt, jt + 128) of segment sg into `dst`, all on barrier `fb`. Paged halves that lie
 // wholly past the segment's keys read the segment's last page instead (their rows are never
-// used), so no block-table entry beyond the sequence is touched.
+// used), so no block-table entry beyond the sequence is touched. Every key tile is read once
+// per call: contiguous loads carry an L2 evict-first policy.
 template <bool PAGED>
 __device__ __forceinline__ void load_kv_tile(const Problem& p, const Segment& sg,
                                              const CUtensorMap* map, uint32_t dst, uint32_t fb,
-                                             int jt) {
+                                             int jt, uint64_t policy) {
   if (!PAGED) {
     const int row = (sg.b * p.Hkv + sg.h) * p.S + jt;
-    tma_load_2d(dst, map, fb, 0, row);
-    tma_load_2d(dst + kHalfBytes, map, fb, 64, row);
+    tma_load_2d_hint(dst, map, fb, 0, row, policy);
+    tma_load_2d_hint(dst + kHalfBytes, map, fb, 64, row, policy);
     return;
   }
   const int jl = sg.j1 - 1;   // last key of the segment
@@ -293,8 +294,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L.misc + 8);
   float* wmax = reinterpret_cast<float*>(base + L.wmax);
   int* lim_s = reinterpret_cast<int*>(base + L.lim);
-  int* pre = reinterpret_cast<int*>(base + L.pre);
-  int* warp_tot = pre + round_up(p.B + 1, 4);
+  int* pre = reinterpret_cast<int*>(base + L.pre);           // the plan's prefix sums
+  int* pre2 = pre + round_up(p.B + 1, 4);                     // the same after the wait
+  int* warp_tot = pre2 + round_up(p.B + 1, 4);
+  // First segment of this CTA and the plan iterator after it: b, h, n, w, j0, j1, whole, slot,
+  // have, pos, end, iterator b, iterator h.
+  long long* spec = reinterpret_cast<long long*>(warp_tot + 32);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Ctl ctl{abort_flag, p.hdr, p.wait_limit_ns};
@@ -305,10 +310,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmo)) : "memory");
   }
 
-  // Q rows R..NQ-1 must read as zero: clear both Q buffers once (TMA rewrites rows < R).
-  for (int i = tid; i < 4 * kQHalf / 16; i += kThreadsTc)
-    reinterpret_cast<uint4*>(base + L.q)[i] = make_uint4(0u, 0u, 0u, 0u);
-  if (tid == 0) {
+  // Q rows R..NQ-1 must read as zero: clear them in both Q buffers once (TMA writes only rows
+  // < R, so no generic store ever meets a copy in flight).
+  {
+    const int per_half = (NQ - p.R) * 8;   // 16-byte chunks of rows [R, NQ) in one half
+    for (int i = tid; i < 4 * per_half; i += kThreadsTc) {
+      const int half = i / per_half, c = i - half * per_half;
+      reinterpret_cast<uint4*>(base + L.q + half * kQHalf + p.R * 128)[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();
+  }
+  auto init_barriers = [&]() {
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
@@ -329,8 +341,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     mbar_init(bar(kBarDrain), 1);
     for (int s = 0; s < kKStages; ++s) mbar_init(bar(kBarKRaw + s), 1);
     for (int s = 0; s < kMaxVStages; ++s) mbar_init(bar(kBarVRaw + s), 1);
-    *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  };
+  if (tid == 0) {
+    init_barriers();
+    *abort_flag = 0;
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -338,84 +353,134 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // Before the wait (small batches, contiguous caches): guess this CTA's first key tiles from
-  // the current seq_lens and have them and Q fetched into L2 while the previous kernel
-  // finishes. The guess is only a hint: the reads bypass L1 (so no stale line can be hit
-  // after the wait), a wrong guess only wastes the prefetch, and the plan is made again from
-  // the values read after the wait.
-  if (!PAGED && warp == 0 && p.B <= 32) {
-    int u = 0;
-    if (lane < p.B) {
-      const int P = __ldcg(p.seq_lens + lane);
-      const int w = p.window_lens ? __ldcg(p.window_lens + lane) : p.W;
-      u = plan_units_of(p, visible_of(p, P, w));
-    }
-    int incl = u;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int excl = incl - u;
-    const long long Tg = (long long)p.Hkv * __shfl_sync(0xffffffffu, incl, 31);
-    const long long pos = Tg > 0 ? plan_lo(p, Tg, blockIdx.x) : 0;
-    const long long Cg = Tg > 0 ? plan_lo(p, Tg, blockIdx.x + 1) - pos : 0;   // units of this CTA
-    const unsigned starts = __ballot_sync(0xffffffffu, lane < p.B && u > 0 &&
-                                                           (long long)p.Hkv * excl <= pos);
-    const int bb = starts ? 31 - __clz(starts) : 0;
-    const int ub = __shfl_sync(0xffffffffu, u, bb), pb = __shfl_sync(0xffffffffu, excl, bb);
-    if (lane == 0 && Cg > 0 && starts != 0u && ub > 0) {
-      const long long off = pos - (long long)p.Hkv * pb;
-      const int hh = (int)(off / ub);
-      const int t0 = max((int)(off - (long long)hh * ub) - p.seg_units, 0);  // first key tile
-      if (hh < p.Hkv) {
-        tma_prefetch_3d(&tmq, 0, hh * p.G, bb * p.W);
-        tma_prefetch_3d(&tmq, 64, hh * p.G, bb * p.W);
-        const int nt = (int)min((long long)(ub - p.seg_units - t0), min(Cg, 2LL));
-        for (int t = 0; t < nt; ++t) {
-          const int row = (bb * p.Hkv + hh) * p.S + (t0 + t) * kNT;
-          tma_prefetch_2d(&tmk, 0, row);
-          tma_prefetch_2d(&tmk, 64, row);
-          tma_prefetch_2d(&tmv, 0, row);
-          tma_prefetch_2d(&tmv, 64, row);
-        }
+  // The plan before the wait (speculative). Made from seq_lens / window_lens as they are now,
+  // read through L2 only, while the previous kernel of the stream finishes: the prefix sums,
+  // this CTA's first segment (thread 0, shared through shared memory so that every role
+  // sees the same values) and, for contiguous caches, an L2 prefetch of its Q and first key
+  // tiles. Right after the wait the producers issue the copies of that first segment, and
+  // the plan is made again from the values read after the wait. If anything the first
+  // segment depends on differs (the prefix sums, or the prefix and window length of its
+  // sequence), the producers drain those copies, the barriers are initialised again and the
+  // kernel continues from the new plan; otherwise the copies are already in flight.
+  plan_prefix<true>(p, pre, warp_tot);
+  long long T = (long long)p.Hkv * pre[p.B];
+  if (tid == 0) {
+    SegmentIter it0 = plan_begin(p, pre, blockIdx.x, T);
+    Segment s0{};
+    const bool have0 = it0.next<true>(p, pre, blockIdx.x, s0);
+    spec[0] = s0.b; spec[1] = s0.h; spec[2] = s0.n; spec[3] = s0.w; spec[4] = s0.j0;
+    spec[5] = s0.j1; spec[6] = s0.whole; spec[7] = s0.slot; spec[8] = have0;
+    spec[9] = it0.pos; spec[10] = it0.end; spec[11] = it0.b; spec[12] = it0.h;
+    if (!PAGED && have0) {
+      // L2 hint only (no shared memory written, no barrier): Q and the first two key tiles.
+      tma_prefetch_3d(&tmq, 0, s0.h * p.G, s0.b * p.W);
+      tma_prefetch_3d(&tmq, 64, s0.h * p.G, s0.b * p.W);
+      const int nt = min(tiles_of(s0), 2);
+      for (int t = 0; t < nt; ++t) {
+        const int row = (s0.b * p.Hkv + s0.h) * p.S + s0.j0 + t * kNT;
+        tma_prefetch_2d(&tmk, 0, row);
+        tma_prefetch_2d(&tmk, 64, row);
+        tma_prefetch_2d(&tmv, 0, row);
+        tma_prefetch_2d(&tmv, 64, row);
       }
     }
   }
+  __syncthreads();
+  Segment sg0;
+  sg0.b = (int)spec[0]; sg0.h = (int)spec[1]; sg0.n = (int)spec[2]; sg0.w = (int)spec[3];
+  sg0.j0 = (int)spec[4]; sg0.j1 = (int)spec[5]; sg0.whole = spec[6] != 0; sg0.slot = (int)spec[7];
+  bool have0 = spec[8] != 0;
   // Everything above is on-chip (or an L2 hint); from here on global memory written by the
   // previous kernel of the stream is read. The merge kernel after this one may start only
   // once every CTA is past the wait (it reads seq_lens before its own wait).
   pdl_wait();
   pdl_trigger();
-  if (tid == 0) {
-    // The tensor maps' descriptors again, now that the wait is over (the copies of the first
-    // tiles are issued right after the plan).
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmq)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+  const uint64_t kv_policy = l2_policy_evict_first();
+  // Speculative copies of the first segment's Q and first key tile (on the barriers the
+  // producers would use for them).
+  bool spec_issued = false;
+  if ((warp == 0 || warp == 6) && lane == 0 && have0) {
+    int w0 = 0, w1 = 0;
+    if (warp == 0) {
+      mbar_expect_tx(bar(kBarQFull), 2u * p.R * 128u);
+      tma_load_3d(sQ, &tmq, bar(kBarQFull), 0, sg0.h * p.G, sg0.b * p.W);
+      tma_load_3d(sQ + kQHalf, &tmq, bar(kBarQFull), 64, sg0.h * p.G, sg0.b * p.W);
+      const bool fuse = p.k_new != nullptr && tile_window(p, sg0, sg0.j0, w0, w1);
+      const uint32_t fb = bar(fuse ? kBarKRaw : kBarKFull);
+      mbar_expect_tx(fb, (uint32_t)kTileBytes);
+      load_kv_tile<PAGED>(p, sg0, &tmk, sK, fb, sg0.j0, kv_policy);
+    } else {
+      const bool fuse = p.v_new != nullptr && tile_window(p, sg0, sg0.j0, w0, w1);
+      const uint32_t fb = bar(fuse ? kBarVRaw : kBarVFull);
+      mbar_expect_tx(fb, (uint32_t)kTileBytes);
+      load_kv_tile<PAGED>(p, sg0, &tmv, sV, fb, sg0.j0, kv_policy);
+    }
+    spec_issued = true;
   }
-  plan_prefix(p, pre, warp_tot);
+  // The plan again, from the values as they are after the wait.
+  plan_prefix<false>(p, pre2, warp_tot);
+  bool differs = false;
+  for (int b = tid; b <= p.B; b += kThreadsTc) differs |= pre[b] != pre2[b];
+  if (tid == 0 && have0)
+    differs |= load_len(p.seq_lens + sg0.b) != sg0.n - sg0.w || window_of(p, sg0.b) != sg0.w;
+  if (p.stall_test & 2) differs = true;   // self-test of the path below
+  if (__syncthreads_or(differs)) {
+    // Rare: the first segment changed. Drain the speculative copies, start the barriers
+    // afresh and take the plan made after the wait.
+    if (spec_issued) {
+      int w0 = 0, w1 = 0;
+      if (warp == 0) {
+        mbar_drain(bar(kBarQFull), 0, 100000000LL);
+        const bool fuse = p.k_new != nullptr && tile_window(p, sg0, sg0.j0, w0, w1);
+        mbar_drain(bar(fuse ? kBarKRaw : kBarKFull), 0, 100000000LL);
+      } else {
+        const bool fuse = p.v_new != nullptr && tile_window(p, sg0, sg0.j0, w0, w1);
+        mbar_drain(bar(fuse ? kBarVRaw : kBarVFull), 0, 100000000LL);
+      }
+      spec_issued = false;
+    }
+    __syncthreads();
+    for (int b = tid; b <= p.B; b += kThreadsTc) pre[b] = pre2[b];
+    if (tid == 0) {
+      for (int i = 0; i < kNumBars; ++i) mbar_inval(bar(i));
+      init_barriers();
+      T = (long long)p.Hkv * pre2[p.B];
+      SegmentIter it0 = plan_begin(p, pre2, blockIdx.x, T);
+      Segment s0{};
+      const bool h0 = it0.next(p, pre2, blockIdx.x, s0);
+      spec[0] = s0.b; spec[1] = s0.h; spec[2] = s0.n; spec[3] = s0.w; spec[4] = s0.j0;
+      spec[5] = s0.j1; spec[6] = s0.whole; spec[7] = s0.slot; spec[8] = h0;
+      spec[9] = it0.pos; spec[10] = it0.end; spec[11] = it0.b; spec[12] = it0.h;
+    }
+    __syncthreads();
+    T = (long long)p.Hkv * pre[p.B];
+    sg0.b = (int)spec[0]; sg0.h = (int)spec[1]; sg0.n = (int)spec[2]; sg0.w = (int)spec[3];
+    sg0.j0 = (int)spec[4]; sg0.j1 = (int)spec[5]; sg0.whole = spec[6] != 0; sg0.slot = (int)spec[7];
+    have0 = spec[8] != 0;
+  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const long long T = (long long)p.Hkv * pre[p.B];
   if (blockIdx.x == 0) {
     for (int i = tid; i <= p.B; i += kThreadsTc) p.pre_g[i] = pre[i];
   }
+  // Every role starts from the first segment above and continues the plan after it.
+  SegmentIter it0;
+  it0.pos = spec[9]; it0.end = spec[10]; it0.b = (int)spec[11]; it0.h = (int)spec[12];
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer: Q, K
     // Lane 0 issues the copies; the whole warp moves the window rows of a fused append.
-    SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
-    Segment sg;
+    SegmentIter it = it0;
+    Segment sg = sg0;
     int g = 0, nseg = 0;
     uint32_t raw_par = 0;   // phase parity of each stage's fused-append barrier
     bool ok = true;
-    while (ok && it.next(p, pre, blockIdx.x, sg)) {
-      if (lane == 0) {
+    for (bool have = have0; ok && have; have = it.next(p, pre, blockIdx.x, sg)) {
+      if (lane == 0 && !(spec_issued && nseg == 0)) {
         const int qs = nseg % qbufs, qu = nseg / qbufs;
         if (qu > 0 && !mbar_wait(bar(kBarQEmpty + qs), (qu - 1) & 1, ctl)) {
           ok = false;
@@ -434,14 +499,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const int ks = g % kKStages, ku = g / kKStages;
         int w0 = 0, w1 = 0;
         const bool fuse = p.k_new != nullptr && tile_window(p, sg, jt, w0, w1);
-        if (lane == 0) {
+        if (lane == 0 && !(spec_issued && g == 0)) {
           if (ku > 0 && !mbar_wait(bar(kBarKEmpty + ks), (ku - 1) & 1, ctl)) {
             ok = false;
           } else {
             const uint32_t dk = sK + ks * kTileBytes;
             const uint32_t fb = bar((fuse ? kBarKRaw : kBarKFull) + ks);
             mbar_expect_tx(fb, (uint32_t)kTileBytes);
-            load_kv_tile<PAGED>(p, sg, &tmk, dk, fb, jt);
+            load_kv_tile<PAGED>(p, sg, &tmk, dk, fb, jt, kv_policy);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -476,26 +541,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------------ TMA producer: V
-    SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
-    Segment sg;
+    SegmentIter it = it0;
+    Segment sg = sg0;
     int g = 0;
     uint32_t raw_par = 0;
     bool ok = true;
-    while (ok && it.next(p, pre, blockIdx.x, sg)) {
+    for (bool have = have0; ok && have; have = it.next(p, pre, blockIdx.x, sg)) {
       const int nt = tiles_of(sg);
       for (int t = 0; t < nt; ++t, ++g) {
         const int jt = sg.j0 + t * kNT;
         const int vs = g % vstages, vu = g / vstages;
         int w0 = 0, w1 = 0;
         const bool fuse = p.v_new != nullptr && tile_window(p, sg, jt, w0, w1);
-        if (lane == 0) {
+        if (lane == 0 && !(spec_issued && g == 0)) {
           if (vu > 0 && !mbar_wait(bar(kBarVEmpty + vs), (vu - 1) & 1, ctl)) {
             ok = false;
           } else {
             const uint32_t dv = sV + vs * kTileBytes;
             const uint32_t fb = bar((fuse ? kBarVRaw : kBarVFull) + vs);
             mbar_expect_tx(fb, (uint32_t)kTileBytes);
-            load_kv_tile<PAGED>(p, sg, &tmv, dv, fb, jt);
+            load_kv_tile<PAGED>(p, sg, &tmv, dv, fb, jt, kv_policy);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -528,8 +593,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
-      Segment sg;
+      SegmentIter it = it0;
+      Segment sg = sg0;
       int g = 0, nseg = 0;
       bool ok = true;
       uint32_t sQseg = sQ;   // Q buffer of the current segment
@@ -552,7 +617,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           umma(tmem + kColO, sdesc(vb + kk * 2048, kHalfBytes, 1024, 2), pdesc, kIdescPV, acc);
         }
       };
-      while (ok && it.next(p, pre, blockIdx.x, sg)) {
+      for (bool have = have0; ok && have; have = it.next(p, pre, blockIdx.x, sg)) {
         const int nt = tiles_of(sg);
         const int qs = nseg % qbufs;
         if (!mbar_wait(bar(kBarQFull + qs), (nseg / qbufs) & 1, ctl)) { ok = false; break; }
@@ -583,7 +648,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
               issue_qk(gq);
               // (Self-test of the failure detection: the first completion is withheld, so the
               // softmax warps' bounded wait for it runs out.)
-              if (!(p.stall_test && gq == 0)) umma_commit(bar(kBarSFull + gq % kSB));
+              if (!((p.stall_test & 1) && gq == 0)) umma_commit(bar(kBarSFull + gq % kSB));
               umma_commit(bar(kBarKEmpty + gq % kKStages));
               if (nqk == nt - 1) umma_commit(bar(kBarQEmpty + qs));
               ++nqk;
@@ -640,11 +705,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     float* rowst = reinterpret_cast<float*>(base + L.mref);   // [2][NQ]
     float* alpha_s = reinterpret_cast<float*>(base + L.alpha); // [NQ]
     const float c2 = p.scale_log2;
-    SegmentIter it = plan_begin(p, pre, blockIdx.x, T);
-    Segment sg;
+    SegmentIter it = it0;
+    Segment sg = sg0;
     int g = 0;
     bool ok = true;
-    while (ok && it.next(p, pre, blockIdx.x, sg)) {
+    for (bool have = have0; ok && have; have = it.next(p, pre, blockIdx.x, sg)) {
       const int nt = tiles_of(sg);
       for (int q = stid; q < NQ; q += 128) {
         if (CAUSAL) lim_s[2 * NQ + q] = (q < p.R) ? min(row_limit(p, sg.n, sg.w, q), sg.j1) : 0;
@@ -919,7 +984,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       } else {
         // A partial goes straight from registers to its slot: for each row the warp writes
         // 32 consecutive channels (128 bytes), with no staging, barrier or copy to wait for.
+        // The merge reads it back after this kernel: kept in L2 (evict-last) while the rest of
+        // the K/V stream passes through.
         float* accp = slot + 2 * p.rows_pad;
+        const uint64_t keep = l2_policy_evict_last();
 #pragma unroll 1
         for (int c = 0; c < NQ / 16; ++c) {
           float ohi[16], olo[16];
@@ -930,12 +998,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int e = 0; e < 16; ++e) {
             const int q = 16 * c + e;
             if (q >= p.R) break;
-            accp[(size_t)q * kHeadDim + row] = ohi[e] + olo[e];
+            st_global_hint(accp + (size_t)q * kHeadDim + row, ohi[e] + olo[e], keep);
           }
         }
         if (stid < p.R) {
-          slot[stid] = rowst[cur * NQ + stid];
-          slot[p.rows_pad + stid] = lsum[stid];
+          st_global_hint(slot + stid, rowst[cur * NQ + stid], keep);
+          st_global_hint(slot + p.rows_pad + stid, lsum[stid], keep);
         }
       }
       // O, l and the shared per-segment buffers are reused by the next segment.
@@ -948,6 +1016,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   if (tid == 64) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   tc_fence_before();
   __syncthreads();
+
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

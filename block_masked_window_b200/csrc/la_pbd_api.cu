@@ -483,6 +483,23 @@ la_status la_pbd_selftest_timeout(const la_pbd_cfg* cfg, const void* q, const vo
                      nullptr, stream, Paging(), t);
 }
 
+la_status la_pbd_selftest_replan(const la_pbd_cfg* cfg, const void* q, const void* k_new,
+                                 const void* v_new, void* k_cache, void* v_cache,
+                                 const int32_t* seq_lens, int32_t W, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  la_status st = check_attn_args(cfg, q, k_cache, v_cache, seq_lens, W, out, workspace,
+                                 workspace_bytes);
+  if (st != LA_OK) return st;
+  if ((k_new == nullptr) != (v_new == nullptr)) return LA_ERR_INVALID_ARG;
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16))) return LA_ERR_INVALID_ARG;
+  if (pick_algo(cfg, W * (cfg->num_q_heads / cfg->num_kv_heads)) != LA_ALGO_TCGEN05)
+    return LA_ERR_UNSUPPORTED;
+  Selftest t;
+  t.stall = 2;
+  return attn_launch(cfg, q, k_cache, v_cache, seq_lens, nullptr, W, out, workspace, k_new,
+                     v_new, stream, Paging(), t);
+}
+
 la_status la_pbd_check(void* workspace, void* stream) {
   if (!workspace || !aligned(workspace, 256)) return LA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;

@@ -67,7 +67,8 @@ struct Problem {
   int seg_units;                // plan units charged per (sequence, KV head) besides its tiles
   float scale_log2;             // scale * log2(e)
   long long wait_limit_ns;      // limit of every bounded device-side wait (tcgen05 kernel)
-  int stall_test;               // self-test: the first S^T completion is never signalled
+  int stall_test;               // self-tests: 1 = the first S^T completion is never signalled,
+                                //             2 = the plan made before the wait is rejected
 };
 
 // Launch parameters of the block-causal prefill kernel.
@@ -94,15 +95,24 @@ __device__ inline float* slot_ptr(const Problem& p, int slot) {
   return p.partials + (size_t)slot * slot_floats(p.rows_pad);
 }
 
+// Loads of seq_lens / window_lens. kL2 = true reads through L2 only (ld.global.cg): the only
+// form used before a kernel's dependency wait, so that no L1 line of a value the previous
+// kernel may still write can be hit after the wait. (Host-callable for the plan inspection
+// entry point, where the arrays are host memory.)
+template <bool kL2 = false>
+__host__ __device__ inline int load_len(const int32_t* a) {
+#ifdef __CUDA_ARCH__
+  return kL2 ? __ldcg(a) : __ldg(a);
+#else
+  return *a;
+#endif
+}
+
 // Window length of sequence b (W when all sequences share it).
-// (Host-callable for the plan inspection entry point, where the arrays are host memory.)
+template <bool kL2 = false>
 __host__ __device__ inline int window_of(const Problem& p, int b) {
   if (!p.window_lens) return p.W;
-#ifdef __CUDA_ARCH__
-  return __ldg(p.window_lens + b);
-#else
-  return p.window_lens[b];
-#endif
+  return load_len<kL2>(p.window_lens + b);
 }
 
 // Visible keys P + w of a sequence with prefix P and window w (0 marks an invalid prefix or
@@ -113,13 +123,9 @@ __host__ __device__ inline int visible_of(const Problem& p, int P, int w) {
 }
 
 // Visible keys of sequence b, P_b + W_b.
+template <bool kL2 = false>
 __host__ __device__ inline int visible_len(const Problem& p, int b) {
-#ifdef __CUDA_ARCH__
-  int P = __ldg(p.seq_lens + b);
-#else
-  int P = p.seq_lens[b];
-#endif
-  return visible_of(p, P, window_of(p, b));
+  return visible_of(p, load_len<kL2>(p.seq_lens + b), window_of<kL2>(p, b));
 }
 
 // Key tiles of a sequence with n visible keys.
@@ -137,6 +143,7 @@ __host__ __device__ inline int plan_units_of(const Problem& p, int n) {
 // Block-wide prefix sum of the plan units U_b (plan_units_of) into pre[0..B] (pre[0] = 0,
 // pre[b+1] = U_0 + ... + U_b).
 // Every thread of the block must call it. `warp_tot` needs one int per warp (<= 32).
+template <bool kL2 = false>
 __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
   const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, wid = tid >> 5;
   const int nwarps = (nthr + 31) >> 5;
@@ -144,7 +151,7 @@ __device__ inline void plan_prefix(const Problem& p, int* pre, int* warp_tot) {
   if (tid == 0) pre[0] = 0;
   for (int base = 0; base < p.B; base += nthr) {
     int b = base + tid;
-    int x = (b < p.B) ? plan_units_of(p, visible_len(p, b)) : 0;
+    int x = (b < p.B) ? plan_units_of(p, visible_len<kL2>(p, b)) : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -209,6 +216,7 @@ struct Segment {
 struct SegmentIter {
   long long pos, end;
   int b, h;
+  template <bool kL2 = false>
   __host__ __device__ bool next(const Problem& p, const int* pre, int c, Segment& sg) {
     while (pos < end) {
       int u = pre[b + 1] - pre[b];
@@ -222,8 +230,8 @@ struct SegmentIter {
       const long long lo = pos > t0 ? pos : t0;
       pos = hi;
       if (hi <= t0) continue;  // only fixed-cost units of (b, h) in this CTA
-      const int n = visible_len(p, b);
-      sg.b = b; sg.h = h; sg.n = n; sg.w = window_of(p, b);
+      const int n = visible_len<kL2>(p, b);
+      sg.b = b; sg.h = h; sg.n = n; sg.w = window_of<kL2>(p, b);
       sg.j0 = (int)(lo - t0) * p.unit;
       const int e = (int)(hi - t0) * p.unit;
       sg.j1 = e < n ? e : n;

@@ -107,7 +107,8 @@ int32_t la_pbd_algo(const la_pbd_cfg* cfg, int32_t window_len);
 /*
  * Bytes of device workspace la_pbd_attn / la_pbd_step need for this configuration and window
  * length on the current device: a 256-byte header (sticky error flags) followed by the
- * per-split partial results (running max, running sum, unnormalised fp32 output rows).
+ * per-split partial results (running max, running sum, unnormalised fp32 output rows), which
+ * a second (merge) kernel of the same call combines.
  * Returns 0 if the configuration is invalid or unsupported.
  */
 size_t la_pbd_workspace_bytes(const la_pbd_cfg* cfg, int32_t window_len);
@@ -312,6 +313,21 @@ la_status la_pbd_selftest_timeout(const la_pbd_cfg* cfg, const void* q, const vo
                                   const void* v_cache, const int32_t* seq_lens,
                                   int32_t window_len, void* out, void* workspace,
                                   size_t workspace_bytes, int64_t wait_limit_ns, void* stream);
+
+/*
+ * Self-test of the tensor-core kernel's early start (the pages have no counterpart). Before
+ * its dependency wait the kernel makes its split plan from seq_lens as they are then; right
+ * after the wait it issues the copies of its first segment and makes the plan again from the
+ * values after the wait; if the two differ, it drains those copies, initialises its barriers
+ * again and follows the new plan. This call enqueues one call in which the comparison is
+ * forced to fail, so that the second path runs: la_pbd_attn (k_new and v_new NULL) or
+ * la_pbd_step (both given), with the same arguments and results (the same output bits and
+ * caches as the normal call). The configuration must select the tcgen05 kernel.
+ */
+la_status la_pbd_selftest_replan(const la_pbd_cfg* cfg, const void* q, const void* k_new,
+                                 const void* v_new, void* k_cache, void* v_cache,
+                                 const int32_t* seq_lens, int32_t window_len, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Synchronise `stream`, read and clear the workspace's sticky device-side error flags.

@@ -67,3 +67,38 @@ def test_every_sm_allocates_after_timeouts(cuda_lib):
     torch.cuda.synchronize()
     assert bmw.la_pbd_check(ws) == 0
     assert_parity(out.cpu(), oracle_step(li, wi.seq_lens, wi.workload.scale), "after timeouts")
+
+
+@pytest.mark.parametrize("name,fused", [("tiny", False), ("single_image", True),
+                                        ("ragged", True), ("ragged", False)])
+def test_rejected_early_plan_gives_the_same_result(cuda_lib, name, fused):
+    """The attention kernel issues its first copies from a plan made before its dependency
+    wait and checks that plan afterwards. With the check forced to fail, the kernel drains
+    those copies, initialises its barriers again and follows the plan made after the wait:
+    the output and the caches must be bit-identical to a normal call."""
+    wl = workloads.WORKLOADS[name]
+    wi = workloads.generate(wl, layers=1)
+    li = wi.layers[0]
+    cfg = bmw.Config.make(wl.batch, wl.num_q_heads, wl.num_kv_heads, wi.max_seq,
+                          algo=bmw.LA_ALGO_TCGEN05)
+    results = []
+    for replan in (False, True):
+        q, kc, vc, sl = to_dev(li.q), to_dev(li.k_cache), to_dev(li.v_cache), to_dev(wi.seq_lens)
+        kn, vn = to_dev(li.k_new), to_dev(li.v_new)
+        ws = bmw.Workspace(cfg, wl.window)
+        out = torch.full_like(q, float("nan"))
+        if not fused:
+            bmw.la_kv_append(cfg, kn, vn, kc, vc, sl, wl.window)
+        if replan:
+            bmw.la_pbd_selftest_replan(cfg, q, kn if fused else None, vn if fused else None,
+                                       kc, vc, sl, wl.window, out, ws)
+        elif fused:
+            bmw.la_pbd_step(cfg, q, kn, vn, kc, vc, sl, wl.window, out, ws)
+        else:
+            bmw.la_pbd_attn(cfg, q, kc, vc, sl, wl.window, out, ws)
+        torch.cuda.synchronize()
+        assert bmw.la_pbd_check(ws) == 0
+        results.append((out.cpu(), kc.cpu(), vc.cpu()))
+    assert torch.equal(results[0][0], results[1][0])
+    assert torch.equal(results[0][1], results[1][1]) and torch.equal(results[0][2], results[1][2])
+    assert_parity(results[1][0], oracle_step(li, wi.seq_lens, wl.scale), f"re-plan {name}")
