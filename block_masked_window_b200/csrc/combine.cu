@@ -20,42 +20,51 @@ namespace la {
 
 constexpr int kCombineRows = 4;
 constexpr int kCombineMaxSlots = 1024;   // >= partials of one sequence (<= grid size)
-template <int kMerge>   // partials loaded in the first round trip
-__global__ void __launch_bounds__(32 * kCombineRows) pbd_combine_kernel(Problem p) {
-  __shared__ float s_w[kCombineRows][kCombineMaxSlots];
+// kMerge partials are loaded in the first round trip; with kMerge = 4 the kernel needs so few
+// registers that 12 blocks fit on an SM, so a batch of many short split sequences (thousands
+// of rows, two or three partials each) is merged in one wave of blocks.
+template <int kMerge>
+__global__ void __launch_bounds__(32 * kCombineRows, kMerge <= 4 ? 12 : 1) pbd_combine_kernel(Problem p) {
+  __shared__ float s_w[kCombineRows][kCombineMaxSlots];   // (16 KB)
   pdl_trigger();
   const int s = blockIdx.y;            // sequence = b * Hkv + h
   const int b = s / p.Hkv, h = s - b * p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * kCombineRows + warp;
   // The plan of sequence b: its units u, the units pb before it and the total. For a batch of
-  // up to 32 sequences each warp derives it before the dependency wait from seq_lens and
-  // window_lens (L2 reads; the attention kernel before this one does not write them, and it
-  // lets this kernel start only after its own wait, so their last writer has completed).
-  // After the wait only the partials remain to be read. A larger batch reads the prefix
-  // sums that attention CTA 0 published.
+  // up to 256 sequences each warp derives it before the dependency wait from seq_lens and
+  // window_lens, 32 sequences at a time (L2 reads; the attention kernel before this one does
+  // not write them, and it lets this kernel start only after its own wait, so their last
+  // writer has completed). After the wait only the partials remain to be read. A larger batch
+  // reads the prefix sums that attention CTA 0 published.
   int u = 0, pb = 0, ptot = 0, wb = p.W;
-  const bool small = p.B <= 32;
-  if (small) {
-    int x = 0, w = p.W;
-    if (lane < p.B) {
-      const int P = __ldcg(p.seq_lens + lane);
-      if (p.window_lens) w = __ldcg(p.window_lens + lane);
-      x = plan_units_of(p, visible_of(p, P, w));
-    }
-    int incl = x;
+  const bool early = p.B <= 256;
+  if (early) {
+    int carry = 0;
+    for (int b0 = 0; b0 < p.B; b0 += 32) {
+      int x = 0, w = p.W;
+      if (b0 + lane < p.B) {
+        const int P = __ldcg(p.seq_lens + b0 + lane);
+        if (p.window_lens) w = __ldcg(p.window_lens + b0 + lane);
+        x = plan_units_of(p, visible_of(p, P, w));
+      }
+      int incl = x;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b >= b0 && b < b0 + 32) {   // (warp-uniform)
+        u = __shfl_sync(0xffffffffu, x, b - b0);
+        pb = carry + __shfl_sync(0xffffffffu, incl - x, b - b0);
+        wb = __shfl_sync(0xffffffffu, w, b - b0);
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    u = __shfl_sync(0xffffffffu, x, b);
-    pb = __shfl_sync(0xffffffffu, incl - x, b);
-    wb = __shfl_sync(0xffffffffu, w, b);
-    ptot = __shfl_sync(0xffffffffu, incl, 31);
+    ptot = carry;
   }
   pdl_wait();
-  if (!small) {
+  if (!early) {
     pb = p.pre_g[b];
     u = p.pre_g[b + 1] - pb;
     ptot = p.pre_g[p.B];
@@ -161,6 +170,10 @@ cudaError_t launch_combine(const Problem& p, cudaStream_t stream) {
   const long long pieces = tiles < p.num_ctas ? tiles : p.num_ctas;
   if (pieces > 16 && (long long)p.B * p.Hkv <= 4)
     return launch_pdl(pbd_combine_kernel<40>, grid, dim3(32 * kCombineRows), 0, stream, p);
+  // With at least half as many (sequence, KV head) pairs as attention CTAs, a pair spans few
+  // CTAs (a longer one still merges correctly, through the loop past the first batch).
+  if (2LL * p.B * p.Hkv >= p.num_ctas)
+    return launch_pdl(pbd_combine_kernel<4>, grid, dim3(32 * kCombineRows), 0, stream, p);
   return launch_pdl(pbd_combine_kernel<16>, grid, dim3(32 * kCombineRows), 0, stream, p);
 }
 

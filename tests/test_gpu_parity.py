@@ -124,11 +124,12 @@ def test_many_short_sequences(algo):
 
 
 @pytest.mark.parametrize("algo", ALGOS, ids=ALGO_IDS)
-@pytest.mark.parametrize("B", [31, 32, 33])
-def test_merge_plan_paths_at_32_sequences(B, algo):
-    """The merge derives a batch's plan itself for up to 32 sequences (one warp-wide scan of
-    seq_lens) and reads the prefix sums the attention kernel published for more: both sides
-    of that boundary, with whole and split sequences and one empty prefix."""
+@pytest.mark.parametrize("B", [31, 32, 33, 255, 256, 257])
+def test_merge_plan_paths(B, algo):
+    """The merge derives a batch's plan itself for up to 256 sequences (warp-wide scans of
+    seq_lens, 32 sequences at a time, with a carry) and reads the prefix sums the attention
+    kernel published for more: both sides of that boundary and of the 32-sequence chunk, with
+    whole and split sequences and one empty prefix."""
     rng = np.random.default_rng(40 + B)
     prefixes = tuple([0] + [int(x) for x in rng.integers(0, 2000, size=B - 1)])
     wi = workloads.random_case(B, prefixes, 6, seed=40 + B)
