@@ -121,8 +121,8 @@ __host__ __device__ inline TcLayout tc_layout(int nq, int vstages, int qbufs, in
   L.lim = a16(L.wmax + 2 * 4 * nq * 4);     // [3][nq] ints: (unused), output offsets, key limits
   L.mref = a16(L.lim + 3 * nq * 4);         // [2][nq]: per-row references
   L.alpha = a16(L.mref + 2 * nq * 4);       // [nq]: rescale factors of the last reference update
-  L.pre = a16(L.alpha + nq * 4);            // plan: [B+1] twice, 32 ints, first segment (16 x 8 B)
-  L.end = L.pre + (2 * round_up(B + 1, 4) + 32) * 4 + 16 * 8;
+  L.pre = a16(L.alpha + nq * 4);            // plan: [B+1], 32 ints, first segment (16 x 8 B)
+  L.end = L.pre + (round_up(B + 1, 4) + 32) * 4 + 16 * 8;
   return L;
 }
 
@@ -295,8 +295,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   float* wmax = reinterpret_cast<float*>(base + L.wmax);
   int* lim_s = reinterpret_cast<int*>(base + L.lim);
   int* pre = reinterpret_cast<int*>(base + L.pre);           // the plan's prefix sums
-  int* pre2 = pre + round_up(p.B + 1, 4);                     // the same after the wait
-  int* warp_tot = pre2 + round_up(p.B + 1, 4);
+  int* warp_tot = pre + round_up(p.B + 1, 4);
   // First segment of this CTA and the plan iterator after it: b, h, n, w, j0, j1, whole, slot,
   // have, pos, end, iterator b, iterator h.
   long long* spec = reinterpret_cast<long long*>(warp_tot + 32);
@@ -358,10 +357,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   // this CTA's first segment (thread 0, shared through shared memory so that every role
   // sees the same values) and, for contiguous caches, an L2 prefetch of its Q and first key
   // tiles. Right after the wait the producers issue the copies of that first segment, and
-  // the plan is made again from the values read after the wait. If anything the first
-  // segment depends on differs (the prefix sums, or the prefix and window length of its
-  // sequence), the producers drain those copies, the barriers are initialised again and the
-  // kernel continues from the new plan; otherwise the copies are already in flight.
+  // the plan is checked against the values read after the wait. If anything the plan or the
+  // first segment depends on differs (a sequence's number of plan units, or the prefix and
+  // window length of the first segment's sequence), the producers drain those copies, the
+  // barriers are initialised again and the kernel continues from the plan made anew;
+  // otherwise the copies are already in flight.
   plan_prefix<true>(p, pre, warp_tot);
   long long T = (long long)p.Hkv * pre[p.B];
   if (tid == 0) {
@@ -417,16 +417,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     spec_issued = true;
   }
-  // The plan again, from the values as they are after the wait.
-  plan_prefix<false>(p, pre2, warp_tot);
-  bool differs = false;
-  for (int b = tid; b <= p.B; b += kThreadsTc) differs |= pre[b] != pre2[b];
-  if (tid == 0 && have0)
-    differs |= load_len(p.seq_lens + sg0.b) != sg0.n - sg0.w || window_of(p, sg0.b) != sg0.w;
-  if (p.stall_test & 2) differs = true;   // self-test of the path below
+  // Check the plan against the values as they are after the wait: the plan is the same if
+  // every sequence has the same number of plan units (hence the same prefix sums), and the
+  // first segment is the same if its sequence also has the same prefix and window length.
+  // (Later segments read their lengths after the wait in any case.) One read per sequence
+  // and the barrier that also orders the tensor-memory allocation before its use.
+  bool differs = (p.stall_test & 2) != 0;   // (self-test of the path below)
+  for (int b = tid; b < p.B; b += kThreadsTc) {
+    const int w = window_of(p, b);
+    const int n = visible_of(p, load_len(p.seq_lens + b), w);
+    differs |= plan_units_of(p, n) != pre[b + 1] - pre[b];
+    if (have0 && b == sg0.b) differs |= n != sg0.n || w != sg0.w;
+  }
+  fence_async_smem();
+  tc_fence_before();
   if (__syncthreads_or(differs)) {
-    // Rare: the first segment changed. Drain the speculative copies, start the barriers
-    // afresh and take the plan made after the wait.
+    // Rare: the plan changed. Drain the speculative copies, start the barriers afresh and
+    // make the plan from the values read after the wait.
     if (spec_issued) {
       int w0 = 0, w1 = 0;
       if (warp == 0) {
@@ -439,15 +446,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       spec_issued = false;
     }
-    __syncthreads();
-    for (int b = tid; b <= p.B; b += kThreadsTc) pre[b] = pre2[b];
+    plan_prefix<false>(p, pre, warp_tot);   // (starts and ends with a barrier)
     if (tid == 0) {
       for (int i = 0; i < kNumBars; ++i) mbar_inval(bar(i));
       init_barriers();
-      T = (long long)p.Hkv * pre2[p.B];
-      SegmentIter it0 = plan_begin(p, pre2, blockIdx.x, T);
+      T = (long long)p.Hkv * pre[p.B];
+      SegmentIter it0 = plan_begin(p, pre, blockIdx.x, T);
       Segment s0{};
-      const bool h0 = it0.next(p, pre2, blockIdx.x, s0);
+      const bool h0 = it0.next(p, pre, blockIdx.x, s0);
       spec[0] = s0.b; spec[1] = s0.h; spec[2] = s0.n; spec[3] = s0.w; spec[4] = s0.j0;
       spec[5] = s0.j1; spec[6] = s0.whole; spec[7] = s0.slot; spec[8] = h0;
       spec[9] = it0.pos; spec[10] = it0.end; spec[11] = it0.b; spec[12] = it0.h;
@@ -458,9 +464,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     sg0.j0 = (int)spec[4]; sg0.j1 = (int)spec[5]; sg0.whole = spec[6] != 0; sg0.slot = (int)spec[7];
     have0 = spec[8] != 0;
   }
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
