@@ -389,7 +389,7 @@ def measure_prefill(args, device, bmw, torch, barrier, max_over_ranks, T=16384, 
               for _ in range(2)]
     for d in copies:
         d["out"] = torch.empty_like(d["q"])
-    ws = bmw.Workspace(cfg, 1, device=device)
+    ws = bmw.PrefillWorkspace(cfg, T, device=device)
     run = lambda d: bmw.la_block_prefill(cfg, d["q"], d["k_cache"], d["v_cache"], d["seq_lens"],  # noqa: E731
                                           bs, d["out"], ws)
     graphs = [capture(torch, lambda d=d: run(d)) for d in copies]

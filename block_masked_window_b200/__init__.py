@@ -19,8 +19,8 @@ __all__ = [
     "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
     "la_noop_chain", "la_pbd_attn_varwin", "la_pbd_algo", "chosen_algo",
     "la_pbd_selftest_timeout", "la_pbd_selftest_replan",
-    "la_pbd_step_varwin", "la_block_prefill", "la_pbd_attn_paged", "la_pbd_step_paged",
-    "Workspace",
+    "la_pbd_step_varwin", "la_block_prefill", "la_block_prefill_workspace_bytes",
+    "la_pbd_attn_paged", "la_pbd_step_paged", "Workspace", "PrefillWorkspace",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_noop_chain", "la_pbd_algo", "la_pbd_selftest_timeout",
                     "la_pbd_selftest_replan",
                     "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill",
-                    "la_pbd_attn_paged", "la_pbd_step_paged"]
+                    "la_block_prefill_workspace_bytes", "la_pbd_attn_paged", "la_pbd_step_paged"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB: Optional[ctypes.CDLL] = None
@@ -110,6 +110,8 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_step_varwin.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.la_block_prefill.restype = i32
     lib.la_block_prefill.argtypes = [cfgp, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp]
+    lib.la_block_prefill_workspace_bytes.restype = sz
+    lib.la_block_prefill_workspace_bytes.argtypes = [cfgp, i32]
     lib.la_pbd_attn_paged.restype = i32
     lib.la_pbd_attn_paged.argtypes = [cfgp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp, vp, sz, vp]
     lib.la_pbd_step_paged.restype = i32
@@ -178,12 +180,16 @@ def la_pbd_workspace_init(workspace, stream=None) -> None:
                                         _stream(stream)), "la_pbd_workspace_init")
 
 
+def la_block_prefill_workspace_bytes(cfg: Config, t_max: int) -> int:
+    return int(load().la_block_prefill_workspace_bytes(ctypes.byref(cfg), int(t_max)))
+
+
 class Workspace:
     """A device workspace sized by ``la_pbd_workspace_bytes`` (allocated through torch)."""
 
-    def __init__(self, cfg: Config, window_len: int, device=None):
+    def __init__(self, cfg: Config, window_len: int, device=None, nbytes: Optional[int] = None):
         import torch
-        n = la_pbd_workspace_bytes(cfg, window_len)
+        n = la_pbd_workspace_bytes(cfg, window_len) if nbytes is None else int(nbytes)
         if n == 0:
             raise LaError(2, "la_pbd_workspace_bytes")
         self.nbytes = n
@@ -194,6 +200,16 @@ class Workspace:
 
     def data_ptr(self) -> int:
         return int(self.tensor.data_ptr())
+
+
+class PrefillWorkspace(Workspace):
+    """A device workspace sized by ``la_block_prefill_workspace_bytes``."""
+
+    def __init__(self, cfg: Config, t_max: int, device=None):
+        n = la_block_prefill_workspace_bytes(cfg, t_max)
+        if n == 0:
+            raise LaError(2, "la_block_prefill_workspace_bytes")
+        super().__init__(cfg, 1, device=device, nbytes=n)
 
 
 def _shapes(cfg: Config, W: int):
@@ -395,7 +411,8 @@ def la_pbd_step_varwin(cfg: Config, q, k_new, v_new, k_cache, v_cache, seq_lens,
 def la_block_prefill(cfg: Config, q, k_cache, v_cache, seq_lens, block_size: int, out,
                      workspace: Workspace, stream=None) -> None:
     """Block-causal prefill attention: q, out [B, T, Hq, D]; caches [B, Hkv, S, D] holding
-    each sequence's keys in rows [0, T_b); seq_lens = T_b."""
+    each sequence's keys in rows [0, T_b); seq_lens = T_b; workspace from
+    ``PrefillWorkspace(cfg, T)``."""
     B, T = int(q.shape[0]), int(q.shape[1])
     Hq, Hkv, D, S = cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, cfg.max_seq
     _check_tensor(q, "q", "bf16", (B, T, Hq, D))

@@ -376,6 +376,30 @@ la_status la_pbd_step_varwin(const la_pbd_cfg* cfg, const void* q, const void* k
                      nullptr, nullptr, stream);
 }
 
+// Prefill workspace: the header, one flag per 128-row V tile [B, Hkv, ntiles] (int32), then
+// V as fp16 [B, Hkv, Tp, D] at a 1024-byte boundary (Tp = ntiles * 128 >= t_max).
+struct PrefillWs {
+  size_t flags, v16, total;
+  int ntiles, Tp;
+};
+static PrefillWs prefill_ws(const la_pbd_cfg* cfg, int32_t t_max) {
+  PrefillWs w;
+  w.ntiles = (t_max + 127) / 128;
+  w.Tp = w.ntiles * 128;
+  const size_t tiles = (size_t)cfg->batch * cfg->num_kv_heads * w.ntiles;
+  w.flags = (size_t)la::kHeaderBytes;
+  w.v16 = (w.flags + tiles * sizeof(int32_t) + 1023) / 1024 * 1024;
+  w.total = w.v16 + tiles * 128 * (size_t)la::kHeadDim * 2;
+  return w;
+}
+
+size_t la_block_prefill_workspace_bytes(const la_pbd_cfg* cfg, int32_t t_max) {
+  if (check_cfg(cfg, 1) != LA_OK || t_max < 1) return 0;
+  if ((long long)cfg->batch * cfg->num_kv_heads * (((long long)t_max + 127) / 128 * 128) >= (1LL << 31))
+    return 0;
+  return prefill_ws(cfg, t_max).total;
+}
+
 la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                            const void* v_cache, const int32_t* seq_lens, int32_t t_max,
                            int32_t block_size, void* out, void* workspace,
@@ -388,8 +412,11 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
     return LA_ERR_INVALID_ARG;
   if (t_max < 1 || block_size < 1) return LA_ERR_INVALID_ARG;
   if ((long long)cfg->batch * t_max >= (1LL << 31)) return LA_ERR_UNSUPPORTED;
+  if ((long long)cfg->batch * cfg->num_kv_heads * (((long long)t_max + 127) / 128 * 128) >= (1LL << 31))
+    return LA_ERR_UNSUPPORTED;
   if (!workspace || !aligned(workspace, 256)) return LA_ERR_WORKSPACE;
-  if (workspace_bytes < (size_t)la::kHeaderBytes) return LA_ERR_WORKSPACE;
+  const PrefillWs w = prefill_ws(cfg, t_max);
+  if (workspace_bytes < w.total) return LA_ERR_WORKSPACE;
   la::PrefillProblem p;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -407,9 +434,13 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
   p.bs = block_size;
   p.scale_log2 = cfg->scale * 1.4426950408889634f;
   p.wait_limit_ns = la::kDefaultWaitLimitNs;
-  CUtensorMap mq, mk, mv;
-  if (la::make_prefill_maps(p, &mq, &mk, &mv) != cudaSuccess) return LA_ERR_CUDA;
-  cudaError_t e = la::launch_prefill_tc(p, &mq, &mk, &mv, (cudaStream_t)stream);
+  p.v16_ok = reinterpret_cast<int*>(static_cast<char*>(workspace) + w.flags);
+  p.v16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + w.v16);
+  p.ntiles = w.ntiles;
+  p.Tp = w.Tp;
+  CUtensorMap mq, mk, mv, mv16;
+  if (la::make_prefill_maps(p, &mq, &mk, &mv, &mv16) != cudaSuccess) return LA_ERR_CUDA;
+  cudaError_t e = la::launch_prefill_tc(p, &mq, &mk, &mv, &mv16, (cudaStream_t)stream);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 

@@ -16,6 +16,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace la {
@@ -83,6 +84,12 @@ struct PrefillProblem {
   int bs;                       // block size of the block mask
   float scale_log2;
   long long wait_limit_ns;      // limit of every bounded device-side wait
+  // V as fp16 (workspace): [B, Hkv, Tp, D], rows [0, T_b) of each (sequence, KV head), and one
+  // flag per 128-row tile, [B, Hkv, ntiles]: 1 when the tile converted exactly enough for the
+  // fp16 product (see prefill_v16_kernel).
+  __half* v16;
+  int* v16_ok;
+  int Tp, ntiles;               // Tp = ntiles * 128 >= T
 };
 
 __host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }

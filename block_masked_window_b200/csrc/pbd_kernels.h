@@ -46,8 +46,9 @@ cudaError_t launch_attn_tc(const Problem& p, const void* tmap_k, const void* tma
 
 // tcgen05 + TMA block-causal prefill (one CTA per 128 query rows of a (sequence, head)).
 size_t prefill_smem_bytes();
+// Launches the V conversion (prefill_v16_kernel) and then the prefill kernel.
 cudaError_t launch_prefill_tc(const PrefillProblem& p, const void* tmap_q, const void* tmap_k,
-                              const void* tmap_v, cudaStream_t stream);
+                              const void* tmap_v, const void* tmap_v16, cudaStream_t stream);
 
 // Merge of the per-split partials into the bf16 output.
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream);

@@ -17,14 +17,21 @@
 // from TMEM, keeps its lazy reference maximum (raised only when a score exceeds it by 2^8;
 // the warp then rescales its O_h rows after the previous PV product has completed) and row
 // sum in registers, and writes its half of the row of P back into tensor memory, over the
-// 64 score columns it has just read: P is written as two bf16 parts, P = P_hi + P_lo (P_lo =
-// bf16(P - P_hi), residual ~2^-17 P), packed two keys per column (P_hi in the first 32
-// columns, P_lo in the next 32), and each PV product is issued for both parts with A read
-// from tensor memory, so the product keeps fp32-level accuracy in P: a single bf16 rounding
-// of P would add a relative L2 error of ~1e-3 to the output, on top of the ~1.7e-3 of its own
-// bf16 rounding. P lives in the S buffer of its tile, so it is double-buffered with S, and
-// shared memory holds only Q and the K and V rings (three stages each). The product S of
-// tile t + 2 reuses that buffer once both halves' PV products of tile t have completed.
+// 64 score columns it has just read, packed two keys per 32-bit column; the PV product reads
+// it there (A from tensor memory). A single bf16 rounding of P would add a relative L2 error
+// of ~1e-3 to the output, on top of the ~1.7e-3 of the output's own bf16 rounding, so P is
+// kept more precisely in one of two ways, chosen per CTA:
+//   * fp16 P (relative rounding 2^-11, 8x finer than bf16) times V converted to fp16 once per
+//     call by prefill_v16_kernel. The conversion is exact for 2^-17 <= |v| <= 65504, so it is
+//     used when every V tile the CTA reads has its largest |v| in [2^-6, 65520) (or is all
+//     zeros): smaller elements then err by at most 2^-25 <= 2^-19 of the tile's largest. One
+//     product per key half and tile.
+//   * otherwise P = P_hi + P_lo, two bf16 parts (P_lo = bf16(P - P_hi), residual ~2^-17 P;
+//     P_hi in the first 32 columns, P_lo in the next 32), each multiplied by the bf16 V tile:
+//     two products per key half and tile.
+// P lives in the S buffer of its tile, so it is double-buffered with S, and shared memory
+// holds only Q and the K and V rings (three stages each). The product S of tile t + 2 reuses
+// that buffer once both halves' PV products of tile t have completed.
 // With no exchange between the halves per tile, the two warps sharing a scheduler drift
 // apart, so one's exponentials overlap the other's maxima and TMEM reads. At the end the pair
 // merges (m, l, O_0, O_1) and each thread normalises and stores 64 of the row's 128 output
@@ -82,8 +89,19 @@ constexpr size_t kPfSmemAlloc = (size_t)kPfSmem + 1024;   // + alignment slack
 // Named barrier 1 over the 256 softmax threads.
 __device__ __forceinline__ void pf_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-// The 64 probabilities of one key half of a row as bf16 P_hi and P_lo, two keys per 32-bit
-// word (the lower key in the low half), into 32 + 32 tensor-memory columns from `taddr`.
+// The 64 probabilities of one key half of a row as fp16, two keys per 32-bit word (the lower
+// key in the low half), into 32 tensor-memory columns from `taddr`.
+__device__ __forceinline__ void store_p16_tmem(uint32_t taddr, const float (&x)[64]) {
+  uint32_t w[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    __half2 h2 = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t*>(&h2);
+  }
+  tmem_st32(taddr, w);
+}
+
+// The same as bf16 P_hi and P_lo, into 32 + 32 tensor-memory columns from `taddr`.
 __device__ __forceinline__ void store_p_tmem(uint32_t taddr, const float (&x)[64]) {
   uint32_t hi[32], lo[32];
 #pragma unroll
@@ -101,9 +119,50 @@ __device__ __forceinline__ void store_p_tmem(uint32_t taddr, const float (&x)[64
 
 }  // namespace
 
+// V rows [0, T_b) of every (sequence, KV head) as fp16 in the workspace, one 128-row tile per
+// block, with the tile's flag: 1 when its largest |v| lies in [2^-6, 65520) or the tile holds
+// only zeros (NaN elements are carried over and do not count), i.e. when the fp16 product
+// is as accurate as the bf16 P_hi + P_lo one (see above). bf16 -> fp16 is exact for
+// 2^-17 <= |v| <= 65504.
+__global__ void __launch_bounds__(256) prefill_v16_kernel(PrefillProblem p) {
+  const int t = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  pdl_wait();   // V and seq_lens may come from the previous kernel of the stream
+  pdl_trigger();
+  int Tb = __ldg(p.seq_lens + b);
+  if (Tb < 0 || Tb > p.T || Tb > p.S) Tb = 0;   // (the attention kernel flags it)
+  const int r0 = t * kBN;
+  const int rows = max(0, min(kBN, Tb - r0));
+  const uint4* src = reinterpret_cast<const uint4*>(p.v + ((size_t)(b * p.Hkv + hk) * p.S + r0) * kHeadDim);
+  uint4* dst = reinterpret_cast<uint4*>(p.v16 + ((size_t)(b * p.Hkv + hk) * p.Tp + r0) * kHeadDim);
+  float vmax = 0.f;
+  for (int c = threadIdx.x; c < rows * (kHeadDim / 8); c += blockDim.x) {
+    const uint4 x = __ldg(src + c);   // 8 bf16
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+      vmax = fmaxf(vmax, fmaxf(fabsf(lo), fabsf(hi)));
+      __half2 h2 = __floats2half2_rn(lo, hi);
+      o[e] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  __shared__ float wmax[8];
+  vmax = warp_max_f32(vmax);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = vmax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
+    p.v16_ok[(size_t)(b * p.Hkv + hk) * p.ntiles + t] = (m < 65520.f && (m >= 0x1p-6f || m == 0.f)) ? 1 : 0;
+  }
+}
+
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                      const __grid_constant__ CUtensorMap tmv, PrefillProblem p) {
+                      const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmv16,
+                      PrefillProblem p) {
   extern __shared__ __align__(1024) char smem_raw[];
   char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(base);
@@ -125,6 +184,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmq)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv16)) : "memory");
     mbar_init(bar(kBQFull), 1);
     for (int s = 0; s < kPfStages; ++s) {
       mbar_init(bar(kBKFull + s), 1);
@@ -148,10 +208,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   pdl_wait();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
   // Tokens of this sequence; an invalid length gives zero rows and the sticky flag.
   int Tb = __ldg(p.seq_lens + b);
@@ -163,6 +219,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int ilast = min(i0 + kBM, Tb) - 1;    // last valid query row of the tile
   const int kmax = (ilast >= i0) ? min(Tb, (ilast / p.bs + 1) * p.bs) : 0;
   const int nk = (kmax + kBN - 1) / kBN;      // key tiles (0: nothing to compute)
+  // fp16 P and V when every V tile this CTA reads converted exactly enough.
+  int ok16 = 1;
+  for (int t = tid; t < nk; t += kPfThreads) ok16 &= __ldcg(p.v16_ok + (size_t)(b * p.Hkv + hk) * p.ntiles + t);
+  tc_fence_before();
+  const bool f16 = __syncthreads_and(ok16) != 0;
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
   if (nk > 0 && warp == 0) {
     // ------------------------------------------------------------------ TMA: Q, K
@@ -190,14 +253,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------------ TMA: V
     if (lane == 0) {
       bool ok = true;
-      const int row0 = (b * p.Hkv + hk) * p.S;
+      // (The fp16 copy has the same layout with Tp rows per (sequence, KV head).)
+      const CUtensorMap* vmap = f16 ? &tmv16 : &tmv;
+      const int row0 = (b * p.Hkv + hk) * (f16 ? p.Tp : p.S);
       int t = 0;
       for (; ok && t < nk; ++t) {
         const int s = t % kPfStages, u = t / kPfStages;
         if (u > 0 && !mbar_wait(bar(kBVEmpty + s), (u - 1) & 1, ctl)) { ok = false; break; }
         mbar_expect_tx(bar(kBVFull + s), (uint32_t)kPTile);
-        tma_load_2d(sV + s * kPTile, &tmv, bar(kBVFull + s), 0, row0 + t * kBN);
-        tma_load_2d(sV + s * kPTile + kPHalf, &tmv, bar(kBVFull + s), 64, row0 + t * kBN);
+        tma_load_2d(sV + s * kPTile, vmap, bar(kBVFull + s), 0, row0 + t * kBN);
+        tma_load_2d(sV + s * kPTile + kPHalf, vmap, bar(kBVFull + s), 64, row0 + t * kBN);
       }
       for (int back = 1; back <= kPfStages && t - back >= 0; ++back) {
         const int tt = t - back;
@@ -209,6 +274,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_f16(128, kBN, 0, 0);     // Q K-major, K K-major
       constexpr uint32_t kIdO = idesc_f16(128, 128, 0, 1);     // P (tensor memory), V MN-major
+      constexpr uint32_t kIdO16 = idesc_f16(128, 128, 0, 1, kOpFp16);   // the same in fp16
       bool ok = mbar_wait(bar(kBQFull), 0, ctl);
       tc_fence_after();
       int nqk = 0, npv[2] = {0, 0};
@@ -239,8 +305,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             prog = true;
           }
         }
-        // O_h += (P_hi + P_lo)_h(t) V_h(t): P columns (keys) [64h, 64h + 64) times V rows
-        // [64h, 64h + 64), once for each bf16 part of P.
+        // O_h += P_h(t) V_h(t): P columns (keys) [64h, 64h + 64) times V rows [64h, 64h + 64),
+        // in fp16, or once for each bf16 part of P.
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int t = npv[hh];
@@ -249,13 +315,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (mbar_test(bar(kBPFull + 2 * hh + (t & 1)), (t >> 1) & 1) &&
                 mbar_test(bar(kBVFull + s), (t / kPfStages) & 1)) {
               tc_fence_after();
-              const uint32_t pa = tmem + kColS + (uint32_t)((t & 1) * kBN + 64 * hh);   // P_hi
+              const uint32_t pa = tmem + kColS + (uint32_t)((t & 1) * kBN + 64 * hh);   // P (P_hi)
               const uint32_t vb = sV + s * kPTile + hh * 4 * 2048;
+              if (f16) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t vd = sdesc(vb + kk * 2048, kPHalf, 1024, 2);
-                umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
-                umma_ts(tmem + kColO + hh * 128, pa + 32 + kk * 8, vd, kIdO, 1u);
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t vd = sdesc(vb + kk * 2048, kPHalf, 1024, 2);
+                  umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vd, kIdO16, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t vd = sdesc(vb + kk * 2048, kPHalf, 1024, 2);
+                  umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+                  umma_ts(tmem + kColO + hh * 128, pa + 32 + kk * 8, vd, kIdO, 1u);
+                }
               }
               umma_commit(bar(kBOFull + 2 * hh + (t & 1)));
               ++npv[hh];
@@ -358,8 +432,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ls[e & 3] += x[e];
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // P_hi and P_lo over this half's scores in the S buffer of the tile (read above).
-      store_p_tmem(s_addr, x);
+      // P (fp16, or P_hi and P_lo) over this half's scores in the S buffer of the tile.
+      if (f16) store_p16_tmem(s_addr, x);
+      else store_p_tmem(s_addr, x);
       tc_wait_st();
       // Keys of this half past the visible range (last tile): zero their V rows so that
       // 0 * x cannot become NaN in the product (those rows may hold anything).
@@ -446,16 +521,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 size_t prefill_smem_bytes() { return kPfSmemAlloc; }
 
 cudaError_t launch_prefill_tc(const PrefillProblem& p, const void* tmap_q, const void* tmap_k,
-                              const void* tmap_v, cudaStream_t stream) {
+                              const void* tmap_v, const void* tmap_v16, cudaStream_t stream) {
   const CUtensorMap& q = *static_cast<const CUtensorMap*>(tmap_q);
   const CUtensorMap& k = *static_cast<const CUtensorMap*>(tmap_k);
   const CUtensorMap& v = *static_cast<const CUtensorMap*>(tmap_v);
+  const CUtensorMap& v16 = *static_cast<const CUtensorMap*>(tmap_v16);
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kPfSmemAlloc);
   if (e != cudaSuccess) return e;
+  e = launch_pdl(prefill_v16_kernel, dim3(p.ntiles, p.Hkv, p.B), dim3(256), 0, stream, p);
+  if (e != cudaSuccess) return e;
   const int ntiles = (p.T + kBM - 1) / kBM;
   return launch_pdl(prefill_tc_kernel, dim3(ntiles, p.Hq, p.B), dim3(kPfThreads), kPfSmemAlloc,
-                    stream, q, k, v, p);
+                    stream, q, k, v, v16, p);
 }
 
 }  // namespace la

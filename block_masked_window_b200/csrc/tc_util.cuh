@@ -23,10 +23,14 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
 
-// Instruction descriptor, kind::f16: D fp32 (bit 4), A and B bf16 (bits 7, 10),
-// A major bit 15, B major bit 16 (1 = MN-major), N >> 3 at bit 17, M >> 4 at bit 24.
-__host__ __device__ constexpr uint32_t idesc_f16(int m, int n, int a_mn, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+// Instruction descriptor, kind::f16: D fp32 (bit 4), the type of A (bits 7-9) and of B (bits
+// 10-12), one value for both (an MMA of this kind takes two operands of the same type):
+// 1 = bf16, 0 = fp16. A major bit 15, B major bit 16 (1 = MN-major), N >> 3 at bit 17,
+// M >> 4 at bit 24.
+constexpr uint32_t kOpBf16 = 1, kOpFp16 = 0;
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n, int a_mn, int b_mn,
+                                                 uint32_t op = kOpBf16) {
+  return (1u << 4) | (op << 7) | (op << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 

@@ -84,9 +84,10 @@ inline cudaError_t make_tma_maps(const Problem& p, TmaMaps* m, long long pool_ro
 }
 
 // Prefill maps: q [B*T rows, Hq, 128] with a box of (64 channels, 1 head, 128 tokens); the K
-// and V caches as for the decode kernel (64 channels x 128 rows), all with the 128-byte swizzle.
+// and V caches as for the decode kernel (64 channels x 128 rows), and the fp16 copy of V
+// [B*Hkv*Tp rows, 128] the same way, all with the 128-byte swizzle.
 inline cudaError_t make_prefill_maps(const PrefillProblem& p, CUtensorMap* mq, CUtensorMap* mk,
-                                     CUtensorMap* mv) {
+                                     CUtensorMap* mv, CUtensorMap* mv16) {
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   {
@@ -109,6 +110,11 @@ inline cudaError_t make_prefill_maps(const PrefillProblem& p, CUtensorMap* mq, C
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   if (enc(mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (void*)p.v, dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  cuuint64_t dims16[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)p.B * p.Hkv * p.Tp};
+  if (enc(mv16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)p.v16, dims16, strides, box, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;

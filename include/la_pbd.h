@@ -234,6 +234,14 @@ la_status la_pbd_step_paged(const la_pbd_cfg* cfg, const void* q, const void* k_
                             size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of device workspace la_block_prefill needs for this configuration and t_max: the
+ * 256-byte header, one int32 per 128-row V tile and an fp16 copy of V
+ * (B * Hkv * ceil(t_max / 128) * 128 rows of D channels, 256 bytes each). Host only.
+ * Returns 0 for an invalid configuration or t_max < 1.
+ */
+size_t la_block_prefill_workspace_bytes(const la_pbd_cfg* cfg, int32_t t_max);
+
+/*
  * Block-causal prefill attention (the block mask of block-diffusion decoding over whole
  * sequences; the PBD window is the last block of it): token i of sequence b attends key j
  * when j <= i or when both lie in the same block of block_size consecutive tokens, i.e. j <
@@ -242,12 +250,18 @@ la_status la_pbd_step_paged(const la_pbd_cfg* cfg, const void* q, const void* k_
  *   k_cache,v_cache bf16 [B, Hkv, S_max, D] with the sequence's keys/values in rows [0, T_b)
  *   seq_lens       device int32 [B]: T_b, 0 <= T_b <= min(t_max, S_max)
  *   block_size     >= 1
- *   workspace      >= 256 bytes (its header, zeroed by la_pbd_workspace_init, receives the
- *                  sticky flags read by la_pbd_check)
- * bf16 inputs, fp32 accumulation, bf16 out; the probabilities enter the PV product as two bf16
- * parts (P_hi + P_lo), which keeps that product at fp32-level accuracy.
+ *   workspace      >= la_block_prefill_workspace_bytes(cfg, t_max), 256-byte aligned (its
+ *                  header, zeroed by la_pbd_workspace_init, receives the sticky flags read by
+ *                  la_pbd_check; the rest needs no initialisation)
+ * bf16 inputs, fp32 accumulation, bf16 out. The probabilities enter the PV product in fp16
+ * (8x finer than bf16), with V converted to fp16 in the workspace first (exact for
+ * 2^-17 <= |v| <= 65504). Where a 128-row V tile that a query tile reads holds a |v| of
+ * 65520 or more, or only values below 2^-6 in magnitude, that query tile uses bf16 V with
+ * the probabilities as two bf16 parts (P_hi + P_lo) instead. Either way the product keeps
+ * fp32-level accuracy in P.
  * A sequence with T_b outside [0, min(t_max, S_max)] gets zero rows and the sticky flag.
- * Asynchronous on `stream`; allocates nothing.
+ * Asynchronous on `stream` (two kernels: the V conversion, then the attention); allocates
+ * nothing.
  */
 la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
                            const void* v_cache, const int32_t* seq_lens, int32_t t_max,

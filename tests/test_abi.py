@@ -125,3 +125,19 @@ def test_algo_choice_without_gpu(lib):
     assert bmw.la_pbd_algo(_cfg(algo=bmw.LA_ALGO_SIMT), 6) == bmw.LA_ALGO_SIMT
     assert lib.la_pbd_algo(ctypes.byref(_cfg()), 17) == -1
     assert lib.la_pbd_algo(ctypes.byref(_cfg(algo=1)), 11) == -2
+
+
+def test_prefill_workspace_layout_without_gpu(lib):
+    # header (256 B), one int32 flag per 128-row V tile, then the fp16 copy of V at a 1024-byte
+    # boundary: B * Hkv * ceil(t_max / 128) * 128 rows of 256 bytes
+    cfg = _cfg(max_seq=16384)
+    tiles = 1 * 2 * 128
+    assert bmw.la_block_prefill_workspace_bytes(cfg, 16384) == 2048 + tiles * 128 * 256
+    assert bmw.la_block_prefill_workspace_bytes(cfg, 1) == 1024 + 2 * 128 * 256
+    assert bmw.la_block_prefill_workspace_bytes(cfg, 0) == 0
+    assert bmw.la_block_prefill_workspace_bytes(_cfg(head_dim=64), 128) == 0
+    # a workspace below that size is rejected on the host, before any CUDA call
+    need = bmw.la_block_prefill_workspace_bytes(cfg, 300)
+    args = (16, 16, 16, 16, 300, 6, 16, 256)
+    assert lib.la_block_prefill(ctypes.byref(cfg), *args, need - 1, None) == 3
+    assert lib.la_block_prefill(ctypes.byref(cfg), *args[:-1], 0, need, None) == 3

@@ -1,12 +1,15 @@
 """GPU parity of the block-causal prefill kernel (la_block_prefill) against the fp64 oracle.
 
 Tolerance: the bar of the whole path, max |gpu - oracle| <= 1e-2 and relative L2 <= 2e-3
-(bf16 in, fp32 accumulate, bf16 out). The kernel splits the probabilities into two bf16 parts
-for the PV product (P = P_hi + P_lo, residual ~2^-17 P), as the decode path does, so the PV
-product adds nothing measurable to the bf16 output rounding (~1.7e-3 relative L2 on N(0,1)
-data). The decode path's extra one-ulp check is not applied: the prefill's 128-key tiles
-change the fp32 summation order over thousands of keys.
+(bf16 in, fp32 accumulate, bf16 out). The PV product takes the probabilities in fp16 with V
+converted to fp16 (exact over the data's range), or, for query tiles that read a V tile
+outside that range, as two bf16 parts (P = P_hi + P_lo, residual ~2^-17 P) times bf16 V.
+Either way the product adds little to the bf16 output rounding (~1.7e-3 relative L2 on
+N(0,1) data); both paths are exercised below. The decode path's extra one-ulp check is not
+applied: the prefill's 128-key tiles change the fp32 summation order over thousands of keys.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -31,7 +34,7 @@ def run_prefill(pi, bs, Hq=16, Hkv=2):
     B, T = pi.q.shape[0], pi.q.shape[1]
     cfg = bmw.Config.make(B, Hq, Hkv, pi.k_cache.shape[2])
     out = torch.full((B, T, Hq, 128), 7.0, dtype=torch.bfloat16, device="cuda")
-    ws = bmw.Workspace(cfg, 1)
+    ws = bmw.PrefillWorkspace(cfg, T)
     bmw.la_block_prefill(cfg, to_dev(pi.q), to_dev(pi.k_cache), to_dev(pi.v_cache),
                          to_dev(pi.seq_lens), bs, out, ws)
     torch.cuda.synchronize()
@@ -101,3 +104,43 @@ def test_prefill_invalid_length_flagged():
     assert bmw.la_pbd_check(ws) == 5
     assert torch.equal(out[1], torch.zeros_like(out[1]))
     check(out[0, :100], oracle_prefill(pi, 0, 6), "valid sequence beside an invalid one")
+
+
+@pytest.mark.parametrize("scale_log2", [17, -12])
+def test_prefill_v_outside_fp16_range(scale_log2):
+    """V scaled by 2^17 (beyond fp16) or 2^-12 (below the fp16 path's lower bound): every
+    query tile takes the bf16 P_hi + P_lo path. Scaling V by a power of two scales the
+    output exactly (no overflow or underflow in bf16), so out * 2^-s must meet the bars
+    against the oracle on the unscaled V."""
+    lens, bs = (300,), 6
+    pi = workloads.prefill_case(lens, seed=73)
+    ref = oracle_prefill(pi, 0, bs)
+    pi.v_cache = pi.v_cache * (2.0 ** scale_log2)
+    out, ws = run_prefill(pi, bs)
+    assert bmw.la_pbd_check(ws) == 0
+    check(out[0, :300].float() * (2.0 ** -scale_log2), ref, f"prefill V x 2^{scale_log2}")
+
+
+def test_prefill_mixed_paths():
+    """One 128-row V tile beyond fp16 (rows [256, 384) x 2^17): the query tiles that read it
+    take the bf16 path, the others the fp16 path, in the same launch. The outputs span five
+    orders of magnitude and some are small sums of large terms, whose fp32 accumulation
+    error scales with the terms, not with the sum. So the bar is relative L2 plus max |err|
+    relative to max(1, sum_j p_ij |v_j|) (the oracle on |V|)."""
+    n, bs = 640, 6
+    pi = workloads.prefill_case((n,), seed=75)
+    pi.v_cache[0, :, 256:384] = pi.v_cache[0, :, 256:384] * 2.0 ** 17
+    out, ws = run_prefill(pi, bs)
+    assert bmw.la_pbd_check(ws) == 0
+    ref = oracle_prefill(pi, 0, bs)
+    mag = oracle_prefill(dataclasses.replace(pi, v_cache=pi.v_cache.abs()), 0, bs)
+    got = out[0, :n].double().numpy()
+    assert np.isfinite(got).all()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    worst = (np.abs(got - ref) / np.maximum(1.0, mag)).max()
+    print(f"[parity] prefill mixed paths: rel_l2={rel:.3e} max_err_over_magnitude={worst:.3e}")
+    assert rel <= REL_L2 and worst <= MAX_ABS
+    # Query rows < 252 (block 6) see only keys [0, 252), none of the scaled rows, so they meet
+    # the absolute bar too: rows [0, 128) from the fp16 path, rows [128, 252) from the bf16
+    # path (their query tile also holds rows that see the scaled tile).
+    check(out[0, :252], ref[:252], "prefill rows before the scaled tile")
