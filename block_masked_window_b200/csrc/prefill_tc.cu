@@ -117,6 +117,26 @@ __device__ __forceinline__ void store_p_tmem(uint32_t taddr, const float (&x)[64
   tmem_st32(taddr + 32, lo);
 }
 
+// Paired fp32 arithmetic (two lanes of a 64-bit register).
+__device__ __forceinline__ uint64_t pack_f32x2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 }  // namespace
 
 // V rows [0, T_b) of every (sequence, KV head) as fp16 in the workspace, one 128-row tile per
@@ -431,13 +451,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // p = 2^(x c2 - m_ref) in fp32 (masked scores are -inf: ex2.approx gives exactly 0 for
       // them), and this tile's part of the row sum.
       const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // (Paired fp32 instructions: one FMA and one add per two scores.)
+      const uint64_t c2v = pack_f32x2(c2, c2), nmv = pack_f32x2(-mref, -mref);
+      uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        x[e] = fast_exp2(fmaf(x[e], c2, -mref));
-        ls[e & 3] += x[e];
+      for (int e = 0; e < 64; e += 2) {
+        float y0, y1;
+        unpack_f32x2(fma_f32x2(pack_f32x2(x[e], x[e + 1]), c2v, nmv), y0, y1);
+        x[e] = fast_exp2(y0);
+        x[e + 1] = fast_exp2(y1);
+        ls[(e >> 1) & 3] = add_f32x2(ls[(e >> 1) & 3], pack_f32x2(x[e], x[e + 1]));
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      float l0, l1, l2, l3, l4, l5, l6, l7;
+      unpack_f32x2(ls[0], l0, l1);
+      unpack_f32x2(ls[1], l2, l3);
+      unpack_f32x2(ls[2], l4, l5);
+      unpack_f32x2(ls[3], l6, l7);
+      l += ((l0 + l1) + (l2 + l3)) + ((l4 + l5) + (l6 + l7));
       // P (fp16, or P_hi and P_lo) over this half's scores in the S buffer of the tile.
       if (f16) store_p16_tmem(s_addr, x);
       else store_p_tmem(s_addr, x);
