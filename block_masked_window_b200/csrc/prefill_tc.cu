@@ -117,6 +117,13 @@ __device__ __forceinline__ void store_p_tmem(uint32_t taddr, const float (&x)[64
   tmem_st32(taddr + 32, lo);
 }
 
+// Maximum of three (one instruction; a NaN operand is ignored, as by fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Paired fp32 arithmetic (two lanes of a 64-bit register).
 __device__ __forceinline__ uint64_t pack_f32x2(float a, float b) {
   uint64_t r;
@@ -417,13 +424,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int e = 0; e < 64; ++e)
           if (j0 + e >= lim) x[e] = -INFINITY;
       }
+      // (Three-input maxima: 36 instructions for the 64 scores.)
       float mp[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mp[u] = x[u];
+      for (int u = 0; u < 8; ++u) mp[u] = fmax3(x[u], x[u + 8], x[u + 16]);
 #pragma unroll
-      for (int e = 8; e < 64; ++e) mp[e & 7] = fmaxf(mp[e & 7], x[e]);
-      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * c2;
+      for (int u = 0; u < 8; ++u) mp[u] = fmax3(mp[u], x[u + 24], x[u + 32]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mp[u] = fmax3(mp[u], x[u + 40], x[u + 48]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mp[u] = fmaxf(mp[u], x[u + 56]);
+      const float mt = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) * c2;
       // Lazy reference: raise it only when a score exceeds it by more than 2^8.
       const bool raise = mt > m_ref + kPfLazy || (m_ref == -INFINITY && mt > -INFINITY);
       float alpha = 1.f;
