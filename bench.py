@@ -56,16 +56,21 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+# The sources the decode attention and merge kernels are compiled from (the stored traffic
+# figures are theirs; the prefill kernel and the host code do not affect them).
+DECODE_SOURCES = ("attn_tc.cu", "combine.cu", "pbd_common.cuh", "pbd_kernels.h", "tc_util.cuh",
+                  "tma_util.h")
+
+
 def kernel_sources_digest():
-    """SHA-256 over the CUDA sources of the library (order fixed), to tell whether a stored
+    """SHA-256 over the decode kernels' CUDA sources (order fixed), to tell whether a stored
     ncu traffic figure was taken on the kernels that run now."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_masked_window_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in DECODE_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
 
 
