@@ -158,16 +158,20 @@ def _stream(stream) -> int:
     return int(torch.cuda.current_stream().cuda_stream)
 
 
+_DTYPES = {}
+
+
 def _check_tensor(t, name, dtype_name, shape=None):
-    import torch
-    dt = {"bf16": torch.bfloat16, "i32": torch.int32}[dtype_name]
-    if t.dtype != dt:
+    if not _DTYPES:
+        import torch
+        _DTYPES.update({"bf16": torch.bfloat16, "i32": torch.int32})
+    if t.dtype is not _DTYPES[dtype_name]:
         raise TypeError(f"{name}: expected {dtype_name}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name}: must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != shape:
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
 
 

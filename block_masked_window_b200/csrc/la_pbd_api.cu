@@ -38,6 +38,62 @@ cudaError_t sm_count(int* out) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Encoded TMA tensor maps of recent calls. Encoding the four maps of a call is host work of
+// the same order as the launches themselves, and a decode loop calls with the same few
+// buffers again and again (one set per layer). A map holds only the addresses, sizes and
+// strides it was made from, all of which are in the key, so an entry is valid for any call
+// with an equal key, on any device.
+struct MapKey {
+  const void* ptr[4];            // k, v, q, out
+  int B, Hq, Hkv, G, W, S;
+  long long pool_rows;
+};
+struct MapEntry {
+  MapKey key;
+  la::TmaMaps maps;
+  bool used;
+};
+constexpr int kMapCache = 128;
+MapEntry g_map_cache[kMapCache];
+int g_map_next = 0;
+std::mutex g_map_mu;
+
+cudaError_t tma_maps_for(const Problem& p, long long pool_rows, la::TmaMaps* out) {
+  MapKey key;
+  std::memset(&key, 0, sizeof(key));   // (padding too: keys are compared bytewise)
+  key.ptr[0] = p.k;
+  key.ptr[1] = p.v;
+  key.ptr[2] = p.q;
+  key.ptr[3] = p.out;
+  key.B = p.B;
+  key.Hq = p.Hq;
+  key.Hkv = p.Hkv;
+  key.G = p.G;
+  key.W = p.W;
+  key.S = p.S;
+  key.pool_rows = pool_rows;
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (const MapEntry& e : g_map_cache) {
+      if (e.used && std::memcmp(&e.key, &key, sizeof(key)) == 0) {
+        *out = e.maps;
+        return cudaSuccess;
+      }
+    }
+  }
+  la::TmaMaps m;
+  const cudaError_t e = la::make_tma_maps(p, &m, pool_rows);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  MapEntry& slot = g_map_cache[g_map_next];
+  g_map_next = (g_map_next + 1) % kMapCache;
+  slot.key = key;
+  slot.maps = m;
+  slot.used = true;
+  *out = m;
+  return cudaSuccess;
+}
+
 la_status check_cfg(const la_pbd_cfg* cfg, int32_t W) {
   if (!cfg) return LA_ERR_INVALID_ARG;
   if (cfg->batch < 1 || cfg->batch > la::kMaxBatch) return LA_ERR_INVALID_ARG;
@@ -226,7 +282,7 @@ la_status attn_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
     la::TmaMaps maps;
     const long long pool_rows =
         pg.block_table ? (long long)pg.num_pages * p.Hkv * pg.page_size : 0;
-    if (la::make_tma_maps(p, &maps, pool_rows) != cudaSuccess) return LA_ERR_CUDA;
+    if (tma_maps_for(p, pool_rows, &maps) != cudaSuccess) return LA_ERR_CUDA;
     p.unit = la::tc_tile_keys();
     p.c_min = 1;
     p.seg_units = 0;
