@@ -61,7 +61,7 @@ namespace {
 using namespace tc;
 
 constexpr int kNT = kTileKeys;          // 128 keys per tile
-constexpr int kSegUnits = 2;            // plan units charged per segment (tc_segment_units)
+constexpr int kSegUnits = 3;            // plan units charged per segment (tc_segment_units)
 constexpr int kKStages = 2;
 constexpr int kSBufs = 4;               // S^T buffers in TMEM (most): QK may run kSBufs-1 tiles ahead
 constexpr int kThreadsTc = 224;

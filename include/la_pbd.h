@@ -276,7 +276,7 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
  * unit per tile. All units are laid end to end, and CTA c of `num_ctas` takes one
  * contiguous run of them; the tiles of a (b, h) in one CTA are a segment (a CTA whose run
  * holds only fixed-cost units of (b, h) gets none of it). The attention kernels use
- * unit_keys = 128, seg_units = 2 (tcgen05 kernel) and unit_keys = 32, seg_units = 0
+ * unit_keys = 128, seg_units = 3 (tcgen05 kernel) and unit_keys = 32, seg_units = 0
  * (CUDA-core kernel); the tcgen05 kernel uses seg_units = 0 when B * Hkv * ceil(S_max / 128)
  * does not exceed its grid (148 CTAs on B200), where every CTA gets at most one tile.
  * Sequences with an invalid prefix length contribute nothing.

@@ -141,9 +141,10 @@ def test_merge_plan_paths(B, algo):
 
 def test_plan_fixed_cost_shapes():
     """34 sequences of 1-3 key tiles in a 1024-row cache: the tcgen05 plan charges each
-    (sequence, KV head) two fixed-cost units, so with two units per CTA some CTAs hold only
-    fixed-cost units (no segment), some start inside them, and the rest split sequences or
-    own them whole. The host view of the same plan confirms that the case has all three."""
+    (sequence, KV head) its fixed-cost units ahead of its tiles, so with two or three units
+    per CTA some CTAs hold only fixed-cost units (no segment), some start inside them, and
+    the rest split sequences or own them whole. The host view of the same plan confirms that
+    the case has all three."""
     rng = np.random.default_rng(0)
     prefixes = tuple(int(x) for x in rng.integers(0, 380, size=34))
     wi = workloads.random_case(34, prefixes, 6, seed=21, max_seq=1024)

@@ -102,7 +102,7 @@ def test_plan_ragged(seed):
 
 
 def test_plan_params():
-    assert bmw.la_pbd_plan_params(bmw.LA_ALGO_TCGEN05) == (128, 2)
+    assert bmw.la_pbd_plan_params(bmw.LA_ALGO_TCGEN05) == (128, 3)
     assert bmw.la_pbd_plan_params(bmw.LA_ALGO_SIMT) == (32, 0)
     with pytest.raises(bmw.LaError):
         bmw.la_pbd_plan_params(bmw.LA_ALGO_AUTO)
