@@ -35,7 +35,9 @@
 // With no exchange between the halves per tile, the two warps sharing a scheduler drift
 // apart, so one's exponentials overlap the other's maxima and TMEM reads. At the end the pair
 // merges (m, l, O_0, O_1) and each thread normalises and stores 64 of the row's 128 output
-// channels.
+// channels. The softmax warps' per-tile instruction stream, not a pipe, sets the pace (no
+// pipe is more than ~40% busy), so it uses paired fp32 instructions (one FMA and one add
+// per two scores) and three-input maxima.
 //
 // Roles (352 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 10 TMA for the V
 // ring, warp 1 TMEM owner and MMA issuer, warps 2..9 softmax (warps w and w + 4 share the TMEM
