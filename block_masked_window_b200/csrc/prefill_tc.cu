@@ -6,21 +6,21 @@
 // blocks this is one key limit per row: row i sees keys [0, min(T, (i / bs + 1) * bs)).
 //
 // One CTA computes 128 query rows of one (sequence, query head) against the keys they may
-// see, flash-attention style, on the tensor cores:
-//   S = Q K^T  (M = 128 query rows, N = 128 keys,     K = 128 channels) -> TMEM fp32, 2 bufs
-//   O += P V   (M = 128 query rows, N = 128 channels, K = 128 keys)     -> TMEM fp32
-// The 128 keys of each tile are split into two halves that are processed independently, as
-// two interleaved split-KV streams: half h's probabilities multiply V rows [64h, 64h + 64)
-// into their own accumulator O_h (TMEM: two S buffers and O_0, O_1 fill the 512 columns),
-// with their own reference maximum and row sum, and the two are merged once at the end. Two
-// softmax threads own query row r (TMEM lane r), one per key half: each reads its 64 scores
-// from TMEM, keeps its lazy reference maximum (raised only when a score exceeds it by 2^8;
-// the warp then rescales its O_h rows after the previous PV product has completed) and row
-// sum in registers, and writes its half of the row of P back into tensor memory, over the
-// 64 score columns it has just read, packed two keys per 32-bit column; the PV product reads
-// it there (A from tensor memory). A single bf16 rounding of P would add a relative L2 error
-// of ~1e-3 to the output, on top of the ~1.7e-3 of the output's own bf16 rounding, so P is
-// kept more precisely in one of two ways, chosen per CTA:
+// see, flash-attention style, on the tensor cores, per tile of 128 keys and per key half h:
+//   S_h = Q K_h^T  (M = 128 query rows, N = 64 keys,       K = 128 channels) -> TMEM fp32
+//   O_h += P_h V_h (M = 128 query rows, N = 128 channels,  K = 64 keys)      -> TMEM fp32
+// The two key halves are processed independently, as two interleaved split-KV streams: half
+// h's probabilities multiply V rows [64h, 64h + 64) into their own accumulator O_h (TMEM: two
+// S buffers and O_0, O_1 fill the 512 columns), with their own reference maximum and row sum,
+// and the two are merged once at the end. Two softmax threads own query row r (TMEM lane r),
+// one per key half: each reads its 64 scores from TMEM, keeps its lazy reference maximum
+// (raised only when a score exceeds it by 2^8; the warp then rescales its O_h rows after the
+// previous PV product has completed) and row sum in registers, and writes its half of the row
+// of P back into tensor memory, over the 64 score columns it has just read, packed two keys
+// per 32-bit column; the PV product reads it there (A from tensor memory). A single bf16
+// rounding of P would add a relative L2 error of ~1e-3 to the output, on top of the ~1.7e-3 of
+// the output's own bf16 rounding, so P is kept more precisely in one of two ways, chosen per
+// CTA:
 //   * fp16 P (relative rounding 2^-11, 8x finer than bf16) times V converted to fp16 once per
 //     call by prefill_v16_kernel. The conversion is exact for 2^-17 <= |v| <= 65504, so it is
 //     used when every V tile the CTA reads has its largest |v| in [2^-6, 65520) (or is all
@@ -30,20 +30,22 @@
 //     P_hi in the first 32 columns, P_lo in the next 32), each multiplied by the bf16 V tile:
 //     two products per key half and tile.
 // P lives in the S buffer of its tile, so it is double-buffered with S, and shared memory
-// holds only Q and the K and V rings (three stages each). The product S of tile t + 2 reuses
-// that buffer once both halves' PV products of tile t have completed.
-// With no exchange between the halves per tile, the two warps sharing a scheduler drift
-// apart, so one's exponentials overlap the other's maxima and TMEM reads. At the end the pair
-// merges (m, l, O_0, O_1) and each thread normalises and stores 64 of the row's 128 output
-// channels. The softmax warps' per-tile instruction stream, not a pipe, sets the pace (no
-// pipe is more than ~40% busy), so it uses paired fp32 instructions (one FMA and one add
-// per two scores) and three-input maxima.
+// holds only Q and the K and V rings (three stages each). S_h of tile t + 2 reuses its
+// columns once PV_h of tile t has completed.
+// Each half has its own S and P barriers, so nothing ties the two halves together until the
+// end: the two softmax warps sharing a scheduler (one per half) drift apart by about half a
+// tile, and one's exponentials overlap the other's maxima, TMEM traffic and waits instead of
+// both queueing on the MUFU at once (measured: the softmax of a tile took ~1200 cycles with
+// the halves apart, ~1750 in step). The price is QK^T as N = 64 products, which keep the
+// tensor core as long as N = 128 ones. At the end the pair merges (m, l, O_0, O_1) and each
+// thread normalises and stores 64 of the row's 128 output channels. The softmax uses paired
+// fp32 instructions (one FMA and one add per two scores) and three-input maxima.
 //
-// Roles (352 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 10 TMA for the V
-// ring, warp 1 TMEM owner and MMA issuer, warps 2..9 softmax (warps w and w + 4 share the TMEM
-// lane quarter w % 4: two warps per scheduler hide each other's latencies). Query tiles are
-// scheduled longest first (the last tiles see the most keys). Every wait is bounded (sticky
-// timeout flag, drain, TMEM freed, return).
+// Roles (384 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 10 TMA for the V
+// ring, warp 1 TMEM owner and QK^T issuer, warp 11 PV issuer, warps 2..9 softmax (warps w and
+// w + 4 share the TMEM lane quarter w % 4, one per key half). Query tiles are scheduled
+// longest first (the last tiles see the most keys). Every wait is bounded (sticky timeout
+// flag, drain, TMEM freed, return).
 #include "pbd_common.cuh"
 #include "pbd_kernels.h"
 #include "tc_util.cuh"
@@ -56,7 +58,7 @@ using namespace tc;
 
 constexpr int kBM = 128;                 // query rows per CTA
 constexpr int kBN = 128;                 // keys per tile
-constexpr int kPfThreads = 352;         // 11 warps
+constexpr int kPfThreads = 384;         // 12 warps
 constexpr int kPfStages = 3;             // K and V ring depth
 constexpr int kPHalf = 128 * 128;        // one 64-column half of a 128-row bf16 tile (16 KB)
 constexpr int kPTile = 2 * kPHalf;       // 32 KB: a 128-row x 128-channel bf16 operand tile
@@ -70,8 +72,8 @@ constexpr int kBKFull = 1;                        // [kPfStages]
 constexpr int kBKEmpty = kBKFull + kPfStages;     // [kPfStages]
 constexpr int kBVFull = kBKEmpty + kPfStages;     // [kPfStages]
 constexpr int kBVEmpty = kBVFull + kPfStages;     // [kPfStages]
-constexpr int kBSFull = kBVEmpty + kPfStages;     // [2]
-constexpr int kBPFull = kBSFull + 2;              // [key half][tile parity], 128 arrivals each
+constexpr int kBSFull = kBVEmpty + kPfStages;     // [key half][tile parity]: S_h of the tile
+constexpr int kBPFull = kBSFull + 4;              // [key half][tile parity], one arrival per warp
 constexpr int kBOFull = kBPFull + 4;              // [key half][tile parity]
 constexpr int kBDrain = kBOFull + 4;
 constexpr int kBNum = kBDrain + 1;
@@ -144,6 +146,28 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+
+
+// Bounded wait of an MMA-issuing thread for one phase of a barrier (hardware-suspended
+// try_wait). The limit is counted in SM clock cycles, a cheap register read (a %globaltimer
+// read costs tens of nanoseconds, on these threads' critical path): limit_ns * 2 cycles last
+// at least limit_ns at the 1.965 GHz maximum SM clock.
+constexpr long long kPfCyclesPerNs = 2;
+__device__ __forceinline__ bool mma_poll(uint32_t bar, uint32_t parity, const Ctl& ctl) {
+  if (mbar_test(bar, parity)) return true;
+  const long long c0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*ctl.abort_flag) return false;
+      if (clock64() - c0 > ctl.limit_ns * kPfCyclesPerNs) {
+        *ctl.abort_flag = 1;
+        atomicOr(&ctl.hdr->err, kErrTimeout);
+        return false;
+      }
+    }
+  }
 }
 
 }  // namespace
@@ -221,12 +245,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(bar(kBVFull + s), 1);
       mbar_init(bar(kBVEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) mbar_init(bar(kBSFull + s), 1);
+    for (int s = 0; s < 4; ++s) mbar_init(bar(kBSFull + s), 1);
     for (int s = 0; s < 4; ++s) {
-      mbar_init(bar(kBPFull + s), 128);
+      mbar_init(bar(kBPFull + s), 4);   // one arrival per softmax warp of the half
       mbar_init(bar(kBOFull + s), 1);
     }
-    mbar_init(bar(kBDrain), 1);
+    mbar_init(bar(kBDrain), 2);   // both issuing threads
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -298,10 +322,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_drain(bar(kBVFull + tt % kPfStages), (tt / kPfStages) & 1, 100000000LL);
       }
     }
-  } else if (nk > 0 && warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (nk > 0 && (warp == 1 || warp == 11)) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Two issuing threads, each in a fixed order: warp 1 issues every QK^T, warp 11 every PV
+    // (each commits and drains its own products). A tcgen05.mma returns to its thread only
+    // at the tensor core's pace (~65 cycles per M128 N128 K16 product, a few queued), so with
+    // one issuer PV(t) queued behind QK^T(t + 1), and QK^T(t + 2) waits for PV(t) (P(t) lives
+    // in S's columns): that chain, not a pipe, set the pace.
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_f16(128, kBN, 0, 0);     // Q K-major, K K-major
+      constexpr uint32_t kIdS64 = idesc_f16(128, 64, 0, 0);    // Q K-major, K K-major, N = 64 keys
       constexpr uint32_t kIdO = idesc_f16(128, 128, 0, 1);     // P (tensor memory), V MN-major
       constexpr uint32_t kIdO16 = idesc_f16(128, 128, 0, 1, kOpFp16);   // the same in fp16
       // Operand descriptors, computed once and advanced by their offsets (the start-address
@@ -309,87 +338,69 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // 256 KB, so adding offset / 16 never carries out of it).
       const uint64_t dq = sdesc(sQ, 16, 1024, 2), dk = sdesc(sK, 16, 1024, 2);
       const uint64_t dv = sdesc(sV, kPHalf, 1024, 2);
-      bool ok = mbar_wait(bar(kBQFull), 0, ctl);
-      tc_fence_after();
-      int nqk = 0, npv[2] = {0, 0};
-      long long t_prog = now_ns();
-      uint32_t spins = 0;
-      while (ok && (npv[0] < nk || npv[1] < nk)) {
-        bool prog = false;
-        // O_h += P_h(t) V_h(t): P columns (keys) [64h, 64h + 64) times V rows [64h, 64h + 64),
-        // in fp16, or once for each bf16 part of P. Issued before the next QK^T: QK^T(t + 2)
-        // waits for PV(t) to complete, so PV(t) must not queue behind another product
-        // (measured: checking QK^T first kept the softmax waiting ~0.5 us per tile).
+      bool ok = true;
+      if (warp == 1) {
+        // S(t) into buffer t & 1 once K(t) has landed and both halves' PV(t - 2) products,
+        // which read P(t - 2) from that buffer, have completed.
+        ok = mma_poll(bar(kBQFull), 0, ctl);
+        for (int t = 0; ok && t < nk; ++t) {
+          const int s = t % kPfStages;
+          ok = mma_poll(bar(kBKFull + s), (t / kPfStages) & 1, ctl);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int t = npv[hh];
-          if (t < nqk) {
-            const int s = t % kPfStages;
-            if (mbar_test(bar(kBPFull + 2 * hh + (t & 1)), (t >> 1) & 1) &&
-                mbar_test(bar(kBVFull + s), (t / kPfStages) & 1)) {
-              tc_fence_after();
-              const uint32_t pa = tmem + kColS + (uint32_t)((t & 1) * kBN + 64 * hh);   // P (P_hi)
-              const uint64_t vb = dv + ((uint32_t)(s * kPTile + hh * 4 * 2048) >> 4);
-              if (f16) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t vd = vb + kk * (2048 >> 4);
-                  umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vd, kIdO16, (t > 0 || kk > 0) ? 1u : 0u);
-                }
-              } else {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t vd = vb + kk * (2048 >> 4);
-                  umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
-                  umma_ts(tmem + kColO + hh * 128, pa + 32 + kk * 8, vd, kIdO, 1u);
-                }
-              }
-              umma_commit(bar(kBOFull + 2 * hh + (t & 1)));
-              ++npv[hh];
-              // The V tile is free once both halves' products of it are issued.
-              if (npv[hh ^ 1] > t) umma_commit(bar(kBVEmpty + s));
-              prog = true;
+          for (int hh = 0; hh < 2; ++hh) {
+            // S_h(t): the scores of key half h (N = 64) into columns [64h, 64h + 64) of the
+            // buffer, once PV_h(t - 2) (which reads P_h(t - 2) from them) has completed.
+            if (t >= 2) {
+              const int tp = t - 2;
+              ok = ok && mma_poll(bar(kBOFull + 2 * hh + (tp & 1)), (tp >> 1) & 1, ctl);
             }
-          }
-        }
-        // S(t) into buffer t & 1 once both halves' PV(t - 2) products, which read P(t - 2)
-        // from that buffer, have completed.
-        if (nqk < nk) {
-          const int s = nqk % kPfStages;
-          const int tp = nqk - 2;
-          const bool sfree = tp < 0 || (mbar_test(bar(kBOFull + (tp & 1)), (tp >> 1) & 1) &&
-                                        mbar_test(bar(kBOFull + 2 + (tp & 1)), (tp >> 1) & 1));
-          if (sfree && mbar_test(bar(kBKFull + s), (nqk / kPfStages) & 1)) {
+            if (!ok) break;
             tc_fence_after();
-            const uint32_t d = tmem + kColS + (uint32_t)((nqk & 1) * kBN);
-            const uint64_t kb = dk + ((uint32_t)(s * kPTile) >> 4);
+            const uint32_t d = tmem + kColS + (uint32_t)((t & 1) * kBN + 64 * hh);
+            const uint64_t kb = dk + ((uint32_t)(s * kPTile + hh * 64 * 128) >> 4);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t off = (uint32_t)((kk >> 2) * kPHalf + (kk & 3) * 32) >> 4;
-              umma(d, dq + off, kb + off, kIdS, kk > 0);
+              umma(d, dq + off, kb + off, kIdS64, kk > 0);
             }
-            umma_commit(bar(kBSFull + (nqk & 1)));
-            umma_commit(bar(kBKEmpty + s));
-            ++nqk;
-            prog = true;
+            umma_commit(bar(kBSFull + 2 * hh + (t & 1)));
           }
+          if (!ok) break;
+          umma_commit(bar(kBKEmpty + s));
         }
-        if (prog) {
-          spins = 0;
-          t_prog = now_ns();
-          continue;
-        }
-        __nanosleep(32);
-        if ((++spins & 63u) == 0) {
-          if (*abort_flag) { ok = false; break; }
-          if (now_ns() - t_prog > p.wait_limit_ns) {
-            *abort_flag = 1;
-            atomicOr(&p.hdr->err, kErrTimeout);
-            ok = false;
-            break;
+      } else {
+        // O_h += P_h(t) V_h(t) for each half as its P lands: P columns (keys) [64h, 64h + 64)
+        // times V rows [64h, 64h + 64), in fp16, or once for each bf16 part of P.
+        for (int t = 0; ok && t < nk; ++t) {
+          const int s = t % kPfStages;
+          ok = mma_poll(bar(kBVFull + s), (t / kPfStages) & 1, ctl);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (!ok) break;
+            ok = mma_poll(bar(kBPFull + 2 * hh + (t & 1)), (t >> 1) & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t pa = tmem + kColS + (uint32_t)((t & 1) * kBN + 64 * hh);   // P (P_hi)
+            const uint64_t vb = dv + ((uint32_t)(s * kPTile + hh * 4 * 2048) >> 4);
+            if (f16) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vb + kk * (2048 >> 4), kIdO16, (t > 0 || kk > 0) ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t vd = vb + kk * (2048 >> 4);
+                umma_ts(tmem + kColO + hh * 128, pa + kk * 8, vd, kIdO, (t > 0 || kk > 0) ? 1u : 0u);
+                umma_ts(tmem + kColO + hh * 128, pa + 32 + kk * 8, vd, kIdO, 1u);
+              }
+            }
+            umma_commit(bar(kBOFull + 2 * hh + (t & 1)));
           }
+          if (!ok) break;
+          umma_commit(bar(kBVEmpty + s));   // the V tile is free once both products complete
         }
       }
+      // Drain this thread's products before TMEM can be released.
       umma_commit(bar(kBDrain));
       mbar_drain(bar(kBDrain), 0, 100000000LL);
     }
@@ -410,7 +421,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int j0 = t * kBN + 64 * half;          // first key of this thread's half
       const uint32_t s_addr = lane_addr + kColS + (uint32_t)((t & 1) * kBN + 64 * half);
       // (Every lane waits on the same barrier; the vote keeps the error path warp-uniform.)
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBSFull + (t & 1)), (t >> 1) & 1, ctl))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(kBSFull + 2 * half + (t & 1)), (t >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       // This half's 64 scores: two 32-column TMEM reads, one wait.
       float x[64];
@@ -499,10 +510,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(0u), "r"(0u),
                        "r"(0u), "r"(0u));
         }
+        // (Only these generic stores need ordering before the async proxy's reads; P went to
+        // tensor memory.)
+        fence_async_smem();
       }
-      fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(kBPFull + 2 * half + (t & 1)));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBPFull + 2 * half + (t & 1)));
     }
     // Epilogue: both halves' last products complete, then the pair merges
     //   M = max(m_0, m_1), a_h = 2^(m_h - M), out = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1)
