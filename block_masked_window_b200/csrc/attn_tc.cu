@@ -912,11 +912,31 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       // is written straight to its slot.
       float* slot = sg.whole ? nullptr : slot_ptr(p, sg.slot);
       const uint32_t stg = sP;
+      const uint64_t keep = l2_policy_evict_last();
+      if (!sg.whole) {
+        // A partial's O is not normalised, so it is written first, straight from registers
+        // to its slot, and its stores drain while the row sums are reduced: for each row the
+        // warp writes 32 consecutive channels (128 bytes). The merge reads it back after this
+        // kernel: kept in L2 (evict-last) while the rest of the K/V stream passes through.
+        float* accp = slot + 2 * p.rows_pad;
+#pragma unroll 1
+        for (int c = 0; c < NQ / 16; ++c) {
+          float ohi[16], olo[16];
+          tmem_ld16(lane_addr + kColO + 16 * c, ohi);
+          tmem_ld16(lane_addr + kColO + NQ + 16 * c, olo);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int q = 16 * c + e;
+            if (q >= p.R) break;
+            st_global_hint(accp + (size_t)q * kHeadDim + row, ohi[e] + olo[e], keep);
+          }
+        }
+      }
       // Row sums: reduce the 128 key lanes' partials, 16 rows at a time. Within a warp a
       // butterfly halves the values each lane holds at every step (16 + 8 + 4 + 2 + 1
       // shuffles leave lane l with the warp's sum of row l & 15); the four warps' sums meet in
       // shared memory.
-      float* lsum = wmax;              // [NQ] row sums of this segment
       float* wsum = wmax + NQ;         // [4][NQ] per-warp sums
 #pragma unroll 1
       for (int c = 0; c < NQ / 16; ++c) {
@@ -939,13 +959,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       softmax_bar();
       float* linv = wmax + 5 * NQ;     // [NQ] reciprocals of the row sums
-      if (stid < NQ) {
-        const float l = (wsum[stid] + wsum[NQ + stid]) + (wsum[2 * NQ + stid] + wsum[3 * NQ + stid]);
-        lsum[stid] = l;
-        linv[stid] = 1.f / l;
-      }
-      softmax_bar();
-      if (sg.whole) {
+      if (!sg.whole) {
+        if (stid < p.R) {
+          const float l = (wsum[stid] + wsum[NQ + stid]) + (wsum[2 * NQ + stid] + wsum[3 * NQ + stid]);
+          st_global_hint(slot + stid, rowst[cur * NQ + stid], keep);
+          st_global_hint(slot + p.rows_pad + stid, l, keep);
+        }
+      } else {
+        if (stid < NQ) {
+          const float l = (wsum[stid] + wsum[NQ + stid]) + (wsum[2 * NQ + stid] + wsum[3 * NQ + stid]);
+          linv[stid] = 1.f / l;
+        }
+        softmax_bar();
         const int rows_w = sg.w * p.G;
 #pragma unroll 1
         for (int c = 0; c < NQ / 16; ++c) {
@@ -983,30 +1008,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           // The staging buffer is reused as P^T by the next segment: wait until it was read.
           asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        }
-      } else {
-        // A partial goes straight from registers to its slot: for each row the warp writes
-        // 32 consecutive channels (128 bytes), with no staging, barrier or copy to wait for.
-        // The merge reads it back after this kernel: kept in L2 (evict-last) while the rest of
-        // the K/V stream passes through.
-        float* accp = slot + 2 * p.rows_pad;
-        const uint64_t keep = l2_policy_evict_last();
-#pragma unroll 1
-        for (int c = 0; c < NQ / 16; ++c) {
-          float ohi[16], olo[16];
-          tmem_ld16(lane_addr + kColO + 16 * c, ohi);
-          tmem_ld16(lane_addr + kColO + NQ + 16 * c, olo);
-          tc_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int q = 16 * c + e;
-            if (q >= p.R) break;
-            st_global_hint(accp + (size_t)q * kHeadDim + row, ohi[e] + olo[e], keep);
-          }
-        }
-        if (stid < p.R) {
-          st_global_hint(slot + stid, rowst[cur * NQ + stid], keep);
-          st_global_hint(slot + p.rows_pad + stid, lsum[stid], keep);
         }
       }
       // O, l and the shared per-segment buffers are reused by the next segment.
