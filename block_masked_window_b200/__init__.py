@@ -18,7 +18,7 @@ __all__ = [
     "la_pbd_workspace_bytes", "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn",
     "la_pbd_step", "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
     "la_noop_chain", "la_pbd_attn_varwin", "la_pbd_algo", "chosen_algo",
-    "la_pbd_selftest_timeout", "la_pbd_selftest_replan",
+    "la_pbd_selftest_timeout", "la_pbd_selftest_replan", "la_block_prefill_selftest_timeout",
     "la_pbd_step_varwin", "la_block_prefill", "la_block_prefill_workspace_bytes",
     "la_pbd_attn_paged", "la_pbd_step_paged", "Workspace", "PrefillWorkspace",
     "EXPORTED_SYMBOLS",
@@ -40,7 +40,7 @@ EXPORTED_SYMBOLS = ["la_version", "la_status_string", "la_pbd_workspace_bytes",
                     "la_pbd_workspace_init", "la_kv_append", "la_pbd_attn", "la_pbd_step",
                     "la_pbd_check", "la_pbd_attn_static", "la_pbd_plan", "la_pbd_plan_params",
                     "la_noop_chain", "la_pbd_algo", "la_pbd_selftest_timeout",
-                    "la_pbd_selftest_replan",
+                    "la_pbd_selftest_replan", "la_block_prefill_selftest_timeout",
                     "la_pbd_attn_varwin", "la_pbd_step_varwin", "la_block_prefill",
                     "la_block_prefill_workspace_bytes", "la_pbd_attn_paged", "la_pbd_step_paged"]
 
@@ -110,6 +110,9 @@ def load() -> ctypes.CDLL:
     lib.la_pbd_step_varwin.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
     lib.la_block_prefill.restype = i32
     lib.la_block_prefill.argtypes = [cfgp, vp, vp, vp, vp, i32, i32, vp, vp, sz, vp]
+    lib.la_block_prefill_selftest_timeout.restype = i32
+    lib.la_block_prefill_selftest_timeout.argtypes = [cfgp, vp, vp, vp, vp, i32, i32, vp, vp, sz,
+                                                      ctypes.c_int64, vp]
     lib.la_block_prefill_workspace_bytes.restype = sz
     lib.la_block_prefill_workspace_bytes.argtypes = [cfgp, i32]
     lib.la_pbd_attn_paged.restype = i32
@@ -428,6 +431,25 @@ def la_block_prefill(cfg: Config, q, k_cache, v_cache, seq_lens, block_size: int
                                    _ptr(seq_lens), T, int(block_size), _ptr(out),
                                    workspace.data_ptr(), workspace.nbytes, _stream(stream)),
            "la_block_prefill")
+
+
+def la_block_prefill_selftest_timeout(cfg: Config, q, k_cache, v_cache, seq_lens, block_size: int,
+                                      out, workspace: Workspace, wait_limit_ns: int,
+                                      stream=None) -> None:
+    """Enqueue the prefill failure-detection self-test (one la_block_prefill whose first S
+    completion of key half 0 is withheld, every wait limited to `wait_limit_ns`);
+    la_pbd_check then gives 6 (LA_ERR_TIMEOUT)."""
+    B, T = int(q.shape[0]), int(q.shape[1])
+    Hq, Hkv, D, S = cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, cfg.max_seq
+    _check_tensor(q, "q", "bf16", (B, T, Hq, D))
+    _check_tensor(k_cache, "k_cache", "bf16", (B, Hkv, S, D))
+    _check_tensor(v_cache, "v_cache", "bf16", (B, Hkv, S, D))
+    _check_tensor(seq_lens, "seq_lens", "i32", (B,))
+    _check_tensor(out, "out", "bf16", (B, T, Hq, D))
+    _check(load().la_block_prefill_selftest_timeout(
+        ctypes.byref(cfg), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), T,
+        int(block_size), _ptr(out), workspace.data_ptr(), workspace.nbytes, int(wait_limit_ns),
+        _stream(stream)), "la_block_prefill_selftest_timeout")
 
 
 def _check_paged(cfg, q, k_pool, v_pool, block_table, seq_lens, W, out):

@@ -456,10 +456,11 @@ size_t la_block_prefill_workspace_bytes(const la_pbd_cfg* cfg, int32_t t_max) {
   return prefill_ws(cfg, t_max).total;
 }
 
-la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
-                           const void* v_cache, const int32_t* seq_lens, int32_t t_max,
-                           int32_t block_size, void* out, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+static la_status prefill_launch(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* seq_lens, int32_t t_max,
+                                int32_t block_size, void* out, void* workspace,
+                                size_t workspace_bytes, void* stream, long long wait_limit_ns,
+                                int stall) {
   la_status st = check_cfg(cfg, 1);
   if (st != LA_OK) return st;
   if (!q || !k_cache || !v_cache || !seq_lens || !out) return LA_ERR_INVALID_ARG;
@@ -489,7 +490,8 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
   p.T = t_max;
   p.bs = block_size;
   p.scale_log2 = cfg->scale * 1.4426950408889634f;
-  p.wait_limit_ns = la::kDefaultWaitLimitNs;
+  p.wait_limit_ns = wait_limit_ns;
+  p.stall_test = stall;
   p.v16_ok = reinterpret_cast<int*>(static_cast<char*>(workspace) + w.flags);
   p.v16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + w.v16);
   p.ntiles = w.ntiles;
@@ -498,6 +500,25 @@ la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_c
   if (la::make_prefill_maps(p, &mq, &mk, &mv, &mv16) != cudaSuccess) return LA_ERR_CUDA;
   cudaError_t e = la::launch_prefill_tc(p, &mq, &mk, &mv, &mv16, (cudaStream_t)stream);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+la_status la_block_prefill(const la_pbd_cfg* cfg, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* seq_lens, int32_t t_max,
+                           int32_t block_size, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return prefill_launch(cfg, q, k_cache, v_cache, seq_lens, t_max, block_size, out, workspace,
+                        workspace_bytes, stream, la::kDefaultWaitLimitNs, 0);
+}
+
+la_status la_block_prefill_selftest_timeout(const la_pbd_cfg* cfg, const void* q,
+                                            const void* k_cache, const void* v_cache,
+                                            const int32_t* seq_lens, int32_t t_max,
+                                            int32_t block_size, void* out, void* workspace,
+                                            size_t workspace_bytes, int64_t wait_limit_ns,
+                                            void* stream) {
+  if (wait_limit_ns < 1000 || wait_limit_ns > la::kDefaultWaitLimitNs) return LA_ERR_INVALID_ARG;
+  return prefill_launch(cfg, q, k_cache, v_cache, seq_lens, t_max, block_size, out, workspace,
+                        workspace_bytes, stream, wait_limit_ns, 1);
 }
 
 static la_status check_paging(const la_pbd_cfg* cfg, int32_t W, const int32_t* block_table,

@@ -84,6 +84,7 @@ struct PrefillProblem {
   int bs;                       // block size of the block mask
   float scale_log2;
   long long wait_limit_ns;      // limit of every bounded device-side wait
+  int stall_test;               // self-test: 1 = the first S_0 completion is never signalled
   // V as fp16 (workspace): [B, Hkv, Tp, D], rows [0, T_b) of each (sequence, KV head), and one
   // flag per 128-row tile, [B, Hkv, ntiles]: 1 when the tile converted exactly enough for the
   // fp16 product (see prefill_v16_kernel).

@@ -363,7 +363,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               const uint32_t off = (uint32_t)((kk >> 2) * kPHalf + (kk & 3) * 32) >> 4;
               umma(d, dq + off, kb + off, kIdS64, kk > 0);
             }
-            umma_commit(bar(kBSFull + 2 * hh + (t & 1)));
+            // (Self-test of the failure detection: the first completion is withheld, so the
+            // half-0 softmax warps' bounded wait for it runs out.)
+            if (!((p.stall_test & 1) && t == 0 && hh == 0)) umma_commit(bar(kBSFull + 2 * hh + (t & 1)));
           }
           if (!ok) break;
           umma_commit(bar(kBKEmpty + s));

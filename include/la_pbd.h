@@ -329,6 +329,21 @@ la_status la_pbd_selftest_timeout(const la_pbd_cfg* cfg, const void* q, const vo
                                   size_t workspace_bytes, int64_t wait_limit_ns, void* stream);
 
 /*
+ * The same self-test for the block-causal prefill kernel: one la_block_prefill in which every
+ * wait gives up after `wait_limit_ns` (1000 .. 2e9 ns) and the QK^T-issuing thread withholds
+ * the completion signal of the first S product of key half 0, so that the wait of that
+ * half's softmax warps runs out. The call's `out` is then undefined; la_pbd_check on the
+ * workspace afterwards returns LA_ERR_TIMEOUT and clears it, and the workspace serves the
+ * next call as usual. Arguments and errors otherwise as la_block_prefill.
+ */
+la_status la_block_prefill_selftest_timeout(const la_pbd_cfg* cfg, const void* q,
+                                            const void* k_cache, const void* v_cache,
+                                            const int32_t* seq_lens, int32_t t_max,
+                                            int32_t block_size, void* out, void* workspace,
+                                            size_t workspace_bytes, int64_t wait_limit_ns,
+                                            void* stream);
+
+/*
  * Self-test of the tensor-core kernel's early start (the pages have no counterpart). Before
  * its dependency wait the kernel makes its split plan from seq_lens as they are then; right
  * after the wait it issues the copies of its first segment and makes the plan again from the

@@ -15,7 +15,7 @@ import torch
 
 import block_masked_window_b200 as bmw
 import workloads
-from gpu_util import assert_parity, oracle_step, to_dev
+from gpu_util import assert_parity, errors, oracle_step, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -102,3 +102,44 @@ def test_rejected_early_plan_gives_the_same_result(cuda_lib, name, fused):
     assert torch.equal(results[0][0], results[1][0])
     assert torch.equal(results[0][1], results[1][1]) and torch.equal(results[0][2], results[1][2])
     assert_parity(results[1][0], oracle_step(li, wi.seq_lens, wl.scale), f"re-plan {name}")
+
+
+def test_prefill_bounded_wait_runs_out_and_context_recovers(cuda_lib):
+    """The block-causal prefill kernel under the same self-test: the QK^T-issuing thread
+    withholds the completion signal of the first S product of key half 0, so that half's
+    softmax wait runs out after 1 ms. The other roles (the second key half, both issuing
+    threads, both producers) must stop at their next bounded wait, drain, free the tensor
+    memory and return with LA_ERR_TIMEOUT raised; the same workspace then serves a normal
+    prefill that matches the oracle."""
+    import numpy as np
+    import oracle
+    lens, bs = (300, 1000), 6
+    pi = workloads.prefill_case(lens, seed=63, t_max=1024)
+    B, T = pi.q.shape[0], pi.q.shape[1]
+    cfg = bmw.Config.make(B, 16, 2, pi.k_cache.shape[2])
+    q, kc, vc, sl = to_dev(pi.q), to_dev(pi.k_cache), to_dev(pi.v_cache), to_dev(pi.seq_lens)
+    ws = bmw.PrefillWorkspace(cfg, T)
+    out = torch.full((B, T, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    t0 = time.perf_counter()
+    bmw.la_block_prefill_selftest_timeout(cfg, q, kc, vc, sl, bs, out, ws, 1_000_000)
+    st = bmw.la_pbd_check(ws)
+    elapsed = time.perf_counter() - t0
+    assert st == LA_ERR_TIMEOUT, bmw.la_status_string(st)
+    assert elapsed < 5.0, elapsed
+    assert bmw.la_pbd_check(ws) == 0          # read and cleared
+
+    out = torch.full((B, T, 16, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    bmw.la_block_prefill(cfg, q, kc, vc, sl, bs, out, ws)
+    torch.cuda.synchronize()
+    assert bmw.la_pbd_check(ws) == 0
+    out = out.cpu()
+    for b, n in enumerate(lens):
+        ids = np.arange(n) // bs
+        k = pi.k_cache[b, :, :n].permute(1, 0, 2)
+        v = pi.v_cache[b, :, :n].permute(1, 0, 2)
+        ref = oracle.block_prefill_attention(pi.q[b, :n], k, v, ids, pi.scale)
+        # (the prefill's bars: max |err| and relative L2; its tiles sum thousands of keys, so
+        # the decode path's one-ulp check does not apply)
+        assert torch.isfinite(out[b, :n]).all()
+        max_abs, rel = errors(out[b, :n], ref)
+        assert max_abs <= 1e-2 and rel <= 2e-3, (max_abs, rel)
