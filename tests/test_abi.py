@@ -117,6 +117,17 @@ def test_selftest_timeout_validates_before_launching(lib):
                                            limit, None) == 1
 
 
+def test_prefill_selftest_timeout_validates_before_launching(lib):
+    cfg = _cfg(max_seq=1024)
+    # wait limits outside [1 us, 2 s] are rejected before any CUDA call
+    for limit in (0, 999, 3_000_000_000):
+        assert lib.la_block_prefill_selftest_timeout(ctypes.byref(cfg), 16, 16, 16, 16, 256, 6,
+                                                     16, 256, 1 << 30, limit, None) == 1
+    # and so are the prefill's own argument errors (a null q), with a valid limit
+    assert lib.la_block_prefill_selftest_timeout(ctypes.byref(cfg), None, 16, 16, 16, 256, 6,
+                                                 16, 256, 1 << 30, 1_000_000, None) == 1
+
+
 def test_algo_choice_without_gpu(lib):
     # kernel choice is host logic: tcgen05 up to 80 rows per KV head, CUDA cores above
     assert bmw.la_pbd_algo(_cfg(), 6) == bmw.LA_ALGO_TCGEN05
