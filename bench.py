@@ -521,6 +521,8 @@ def main():
     ap.add_argument("--no-compare", action="store_true", help="skip the per-kernel timing table")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--no-prefill", action="store_true", help="skip the block-prefill line")
+    ap.add_argument("--prefill-tokens", type=int, default=16384,
+                    help="sequence length of the block-prefill line")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -583,7 +585,7 @@ def main():
         })
 
     prefill = None if args.no_prefill else measure_prefill(args, device, bmw, torch, barrier,
-                                                           max_over_ranks)
+                                                           max_over_ranks, T=args.prefill_tokens)
 
     if rank != 0:
         if world > 1:
