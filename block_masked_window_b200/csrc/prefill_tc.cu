@@ -340,8 +340,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t dv = sdesc(sV, kPHalf, 1024, 2);
       bool ok = true;
       if (warp == 1) {
-        // S(t) into buffer t & 1 once K(t) has landed and both halves' PV(t - 2) products,
-        // which read P(t - 2) from that buffer, have completed.
+        // Per tile, once K(t) has landed: S_0(t), then S_1(t), into buffer t & 1, each after
+        // its own half's PV(t - 2) has completed; then the K tile is released.
         ok = mma_poll(bar(kBQFull), 0, ctl);
         for (int t = 0; ok && t < nk; ++t) {
           const int s = t % kPfStages;
