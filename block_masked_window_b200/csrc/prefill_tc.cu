@@ -37,9 +37,10 @@
 // tile, and one's exponentials overlap the other's maxima, TMEM traffic and waits instead of
 // both queueing on the MUFU at once (measured: the softmax of a tile took ~1200 cycles with
 // the halves apart, ~1750 in step). The price is QK^T as N = 64 products, which keep the
-// tensor core nearly as long as N = 128 ones (53 against 64 cycles each). At the end the pair merges (m, l, O_0, O_1) and each
-// thread normalises and stores 64 of the row's 128 output channels. The softmax uses paired
-// fp32 instructions (one FMA and one add per two scores) and three-input maxima.
+// tensor core nearly as long as N = 128 ones (53 against 64 cycles each). At the end the
+// pair merges (m, l, O_0, O_1) and each thread normalises and stores 64 of the row's 128
+// output channels. The softmax uses paired fp32 instructions (one FMA and one add per two
+// scores) and three-input maxima.
 //
 // Roles (384 threads, 1 CTA per SM): warp 0 TMA for Q and the K ring, warp 10 TMA for the V
 // ring, warp 1 TMEM owner and QK^T issuer, warp 11 PV issuer, warps 2..9 softmax (warps w and
